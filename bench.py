@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Benchmark of the timestep-adaptive masked INT8 linear on B200.
+
+A step is one denoising step of a whole workload: for every block and every linear of the
+block, tasq_linear_forward(x, layer, step) = block-Hadamard INT8 prologue + masked INT8 GEMM,
+with the step's per-layer bit widths read from the device schedule table. Every (block,
+layer) has its own weights and its own activation buffer, so each step streams its whole
+input set from HBM (larger than L2).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload pixart] [--impl tasq|reference]
+
+N > 1 runs under torchrun, one process per GPU, each an independent replica of the whole
+workload (the path shards along tokens with no exchange); the time is the max over ranks.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "masked-INT8 linear TOPS & tokens/s per denoise step; % of B200 INT8 tensor peak"
+# INT8 dense tensor peak = measured BF16 cuBLAS peak x (4.5 POPS INT8 / 2.25 PFLOPS BF16 nominal)
+INT8_OVER_BF16 = 2.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--workload", default="pixart", choices=list(workloads.WORKLOADS))
+    p.add_argument("--impl", default="tasq", choices=["tasq", "reference"])
+    p.add_argument("--out-dtype", default="f16", choices=["f16", "bf16"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile-case", default=None,
+                   help="workload:layer, run a few forwards of one layer (for ncu captures) and exit")
+    p.add_argument("--launches", type=int, default=3)
+    p.add_argument("--bits", type=int, default=None, help="profile case: bit width (default: 5)")
+    return p.parse_args(argv)
+
+
+# ------------------------------------------------------------------------------ peaks, clocks
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [r for r in csv.reader(io.StringIO(self.tmp.read())) if len(r) >= 9]
+        self.tmp.close()
+        os.unlink(self.tmp.name)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ CPU oracle leg
+def oracle_sample(wl, rows: int, seed: int = 0):
+    """Inputs of one block's linears for `rows` token rows, with each layer's bits at step 0."""
+    data = []
+    sched = workloads.schedule(wl)
+    for j, (_, K, N) in enumerate(wl.block_layers):
+        x = workloads.activations(wl, j, M=rows, seed=seed)
+        w, s_w = workloads.weights(wl, j)
+        data.append((x, w, s_w, int(sched[j, 0]), K, N))
+    return data
+
+
+def run_oracle_sample(wl, data):
+    import oracle
+    ops = 0.0
+    for x, w, s_w, bits, K, N in data:
+        oracle.masked_linear(x, w, s_w, bits, wl.hadamard_n)
+        ops += 2.0 * x.shape[0] * N * K
+    return ops
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_baseline(wl, budget_s: float = 12.0, rows: int = 256):
+    data = oracle_sample(wl, rows)
+    t0 = time.perf_counter()
+    ops, reps = 0.0, 0
+    while True:
+        ops += run_oracle_sample(wl, data)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{reps} x one block ({len(wl.block_layers)} linears) of '{wl.name}' on {rows} token rows, "
+                      f"step-0 bits; {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = workloads.WORKLOADS[args.workload]
+    rows = 64
+    data = oracle_sample(wl, rows)
+    for _ in range(args.warmup):
+        run_oracle_sample(wl, data)
+    t0 = time.perf_counter()
+    ops = 0.0
+    for _ in range(args.steps):
+        ops += run_oracle_sample(wl, data)
+    dt = time.perf_counter() - t0
+    value = ops / dt / 1e12
+    sample = (f"each step: one block ({len(wl.block_layers)} linears) of '{wl.name}' on {rows} of its "
+              f"{wl.tokens} token rows, step-0 bits")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / max(args.steps, 1) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "tokens": wl.tokens, "blocks": wl.blocks, "hadamard_n": wl.hadamard_n,
+                   "sample_rows": rows},
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------ GPU leg
+def setup_workload(T, torch, wl, device, out_dtype):
+    """Context with every layer of the workload, one activation buffer per (block, layer),
+    one output buffer per distinct N. Weights and activations drawn on the device."""
+    L = wl.num_layers
+    layers, keep = [], []
+    for l in range(L):
+        _, K, N = wl.layer_shape(l)
+        w, s_w = workloads.weights_torch(wl, l, device)
+        keep.append((w, s_w))
+        layers.append((N, K, w, s_w))
+    stream = torch.cuda.current_stream()
+    ctx = T.tasq_linear_create(layers, wl.steps, wl.hadamard_n, wl.tokens,
+                               T.TASQ_OUT_F16 if out_dtype == "f16" else T.TASQ_OUT_BF16, stream)
+    torch.cuda.synchronize()
+    del keep, layers
+    T.tasq_set_schedule(ctx, workloads.schedule(wl), stream)
+    xs = [workloads.activations_torch(wl, l, device) for l in range(L)]
+    tdt = torch.float16 if out_dtype == "f16" else torch.bfloat16
+    ys = {}
+    for _, _, N in wl.block_layers:
+        if N not in ys:
+            ys[N] = torch.empty((wl.tokens, N), dtype=tdt, device=device)
+    torch.cuda.synchronize()
+    return ctx, xs, ys
+
+
+def run_step(T, ctx, wl, xs, ys, step, stream):
+    M = wl.tokens
+    per = len(wl.block_layers)
+    for l in range(wl.num_layers):
+        _, K, N = wl.block_layers[l % per]
+        T.tasq_linear_forward(ctx, xs[l], M, K, l, step, ys[N], N, stream)
+
+
+def profile_case(args):
+    import torch
+    import timestep_adaptive_bit_b200 as T
+    name, _, lname = args.profile_case.partition(":")
+    wl = workloads.WORKLOADS[name]
+    j = [n for n, _, _ in wl.block_layers].index(lname or wl.block_layers[0][0])
+    _, K, N = wl.layer_shape(j)
+    dev = torch.device("cuda:0")
+    w, s_w = workloads.weights_torch(wl, j, dev)
+    s = torch.cuda.current_stream()
+    ctx = T.tasq_linear_create([(N, K, w, s_w)], 1, wl.hadamard_n, wl.tokens, T.TASQ_OUT_F16, s)
+    bits = 5 if args.bits is None else args.bits
+    T.tasq_set_schedule(ctx, np.array([[bits]], np.uint8), s)
+    x = workloads.activations_torch(wl, j, dev)
+    y = torch.empty((wl.tokens, N), dtype=torch.float16, device=dev)
+    for _ in range(args.launches):
+        T.tasq_linear_forward(ctx, x, wl.tokens, K, 0, 0, y, N, s)
+    torch.cuda.synchronize()
+    st = T.tasq_get_device_status(ctx)
+    print(json.dumps({"profile_case": args.profile_case, "M": wl.tokens, "K": K, "N": N, "bits": bits,
+                      "launches": args.launches, "device_status": st}))
+    return 0 if st == 0 else 1
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    from timestep_adaptive_bit_b200 import build as _build
+    _build.build()
+    import timestep_adaptive_bit_b200 as T
+
+    if args.profile_case:
+        return profile_case(args)
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+
+    wl = workloads.WORKLOADS[args.workload]
+    ctx, xs, ys = setup_workload(T, torch, wl, device, args.out_dtype)
+    stream = torch.cuda.current_stream()
+    L = wl.num_layers
+
+    for i in range(args.warmup):
+        run_step(T, ctx, wl, xs, ys, i % wl.steps, stream)
+    torch.cuda.synchronize()
+    T.tasq_trace_enable(ctx, args.steps * L)
+    sampler = ClockSampler(local_rank)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.2)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        run_step(T, ctx, wl, xs, ys, i % wl.steps, stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if dist is not None:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    trace = T.tasq_trace_read(ctx)
+    status = T.tasq_get_device_status(ctx)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+
+    # ---- end to end through the public API: pinned host input in, host result out, per step
+    e2e = None
+    if not args.no_e2e:
+        first_K = wl.block_layers[0][1]
+        last_N = wl.block_layers[-1][2]
+        x_host = torch.empty((wl.tokens, first_K), dtype=torch.float16, pin_memory=True)
+        x_host.copy_(xs[0].cpu())
+        y_host = torch.empty((wl.tokens, last_N), dtype=ys[last_N].dtype, pin_memory=True)
+        e_steps = max(1, min(args.steps, 50))
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(e_steps):
+            xs[0].copy_(x_host, non_blocking=True)
+            run_step(T, ctx, wl, xs, ys, i % wl.steps, stream)
+            y_host.copy_(ys[last_N], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
+        if dist is not None:
+            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
+        e_ms = float(ems.item())
+        e2e = {"value": world * e_steps * wl.gemm_ops_per_step() / (e_ms / 1e3) / 1e12, "unit": "TOPS",
+               "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+               "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()),
+               "steps": e_steps, "ms_per_step": e_ms / e_steps}
+
+    peaks, peak_kind = load_peaks()
+    int8_burst = peaks["bf16_tflops"] * INT8_OVER_BF16
+    int8_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * INT8_OVER_BF16
+    total_ops = world * args.steps * wl.gemm_ops_per_step()
+    value = total_ops / (ms_max / 1e3) / 1e12
+    ms_per_step = ms_max / args.steps
+    gemm_tops = trace["gemm_ops"] / (trace["gemm_ms"] / 1e3) / 1e12 if trace["gemm_ms"] > 0 else None
+    pro_gbs = trace["prologue_bytes"] / (trace["prologue_ms"] / 1e3) / 1e9 if trace["prologue_ms"] > 0 else None
+
+    if dist is not None:
+        T.tasq_linear_destroy(ctx)
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0 if status == 0 else 1
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl)
+
+    sched = workloads.schedule(wl)
+    mean_bits = float(np.mean(sched[:, [i % wl.steps for i in range(args.steps)]]))
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": wl.name, "tokens": wl.tokens, "blocks": wl.blocks, "schedule_steps": wl.steps,
+                   "hadamard_n": wl.hadamard_n,
+                   "linears": [f"{n}:{K}->{N}" for n, K, N in wl.block_layers],
+                   "out_dtype": args.out_dtype, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2: each step reads its own activations for every (block, linear) "
+                         f"({sum(x.numel() * 2 for x in xs) / 1e9:.2f} GB) and every layer's weights once"},
+        "tokens_per_s_per_step": wl.tokens / (ms_per_step / 1e3) * world,
+        "pct_int8_peak": 100.0 * value / (int8_burst * world),
+        "mean_bits": mean_bits,
+        "bitops_saved_modelled": 1.0 - mean_bits / 8.0,
+        "roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": int8_burst, "unit": "TFLOP/s",
+                     "frac": (gemm_tops / int8_burst) if gemm_tops else None, "traffic": None,
+                     "kernel": "masked_gemm_kernel", "peak_kind": f"INT8 = 2 x {peak_kind} BF16 burst",
+                     "frac_of_sustained": (gemm_tops / int8_sust) if gemm_tops else None},
+        "prologue_roofline": {"bound": "hbm", "achieved": pro_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": (pro_gbs / peaks["hbm_gbs"]) if pro_gbs else None,
+                              "frac_of_8000": (pro_gbs / 8000.0) if pro_gbs else None},
+        "gemm_share_of_step": trace["gemm_ms"] / max(ms, 1e-9) if trace["gemm_ms"] else None,
+        "clocks": clocks,
+        "gpu_launches": 2 * args.steps * L,
+        "device_status": status,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+    }
+    print(json.dumps(line), flush=True)
+    return 0 if status == 0 else 1
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,189 @@
+/*
+ * tasq.h - C ABI of the timestep-adaptive masked INT8 linear layer (B200, sm_100a).
+ *
+ * One shared INT8 weight buffer per layer serves every denoising step; at step t the layer
+ * runs with the k = 8 - bits[layer][step] least-significant bit planes of every weight
+ * cleared, as in TASQ's Temporal-Spatial LSB Mask (TASQ technical summary, section 2,
+ * "Representacao de Peso Compartilhada e Mascaramento de LSB", equation
+ * Q^(t,l) = Q_n - (1 - M_t,l) * LSB; TASQ abstract: "one shared maximum-precision weight
+ * buffer", no per-stage weight copies, no runtime search, switching costs nothing).
+ * Activations are smoothed by a block Hadamard transform and quantized per token to INT8
+ * before an integer GEMM whose result is dequantized by FP scales (HQ-DM technical summary,
+ * sections 2.1 "Mecanismo" / "Eficiencia de Hardware" and 2.2 "Quantizacao Simetrica";
+ * 6Bit-Diffusion section 2.A, Block Hadamard Transform).
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" must be CUDA device (or managed) memory of the device that was
+ *     current when the context was created; "host" pointers are ordinary host memory.
+ *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy default stream.
+ *     Work is enqueued on that stream and the call returns without synchronising unless
+ *     stated otherwise.
+ *   - Every argument is validated on the host before anything is enqueued. On error the call
+ *     enqueues nothing, returns a non-zero tasq_status and records a message readable with
+ *     tasq_last_error() on the calling thread. No call aborts, throws or traps.
+ *   - Layouts are row-major. Alignment: every device pointer 16-byte aligned; every row
+ *     stride (in elements) a multiple of 8 (16 bytes for FP16), so rows stay 16-byte aligned.
+ *   - A context is not thread-safe: one thread (or external locking) per context.
+ */
+#ifndef TASQ_H_
+#define TASQ_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TASQ_OK = 0,
+  TASQ_ERR_INVALID_ARG = 1,      /* a pointer, size, index, alignment or bit width is invalid */
+  TASQ_ERR_CUDA = 2,             /* a CUDA runtime / driver call failed (message has details) */
+  TASQ_ERR_UNSUPPORTED_ARCH = 3, /* the current device is not compute capability 10.0 */
+  TASQ_ERR_WORKSPACE = 4,        /* M exceeds the max_tokens the context was created with */
+  TASQ_ERR_TIMEOUT = 5,          /* a bounded device-side wait gave up (see device status) */
+} tasq_status;
+
+typedef enum {
+  TASQ_OUT_F16 = 0,   /* IEEE binary16 outputs */
+  TASQ_OUT_BF16 = 1,  /* bfloat16 outputs */
+} tasq_out_dtype;
+
+/* Device status bits written by bounded waits that ran out (see tasq_get_device_status). */
+#define TASQ_DEVICE_TIMEOUT_PRODUCER 0x1u
+#define TASQ_DEVICE_TIMEOUT_MMA 0x2u
+#define TASQ_DEVICE_TIMEOUT_MASK 0x4u
+#define TASQ_DEVICE_TIMEOUT_EPILOGUE 0x8u
+#define TASQ_DEVICE_TIMEOUT_DRAIN 0x10u
+#define TASQ_DEVICE_BAD_BITS 0x100u
+
+/* Limits of this implementation. */
+#define TASQ_MAX_KP 16384           /* Kp = ceil(K / n) * n must not exceed this */
+
+/*
+ * One linear layer y = x W^T, described for tasq_linear_create.
+ *   N   : out-features (rows of W), N >= 1.
+ *   K   : in-features (columns of the activations), K >= 8 and K % 8 == 0.
+ *   w   : INT8 weight codes [N, Kp], row-major, Kp = ceil(K / n) * n (n = hadamard_n). The
+ *         codes are read in the Hadamard-rotated input basis (the basis the activations are
+ *         transformed into), so every one of the Kp columns takes part. Host or device
+ *         memory; copied by tasq_linear_create, the caller keeps ownership.
+ *   s_w : FP32 per-output-channel weight scales [N]. Host or device; copied.
+ */
+typedef struct {
+  int32_t N;
+  int32_t K;
+  const int8_t* w;
+  const float* s_w;
+} tasq_layer_desc;
+
+typedef struct tasq_ctx tasq_ctx;
+
+/*
+ * Create a context owning one shared weight buffer for `num_layers` layers, a device schedule
+ * table bits[num_layers][num_steps] (every entry initialised to 8 = full precision), and an
+ * activation workspace for up to `max_tokens` tokens.
+ *   out         : receives the context; *out is set to NULL on failure.
+ *   layers      : host array [num_layers] of layer descriptors.
+ *   hadamard_n  : block size of the Hadamard transform along K, 64 or 128.
+ *   max_tokens  : largest M any later forward may use, >= 1.
+ *   out_dtype   : a tasq_out_dtype for the outputs of tasq_linear_forward.
+ *   stream      : stream used for the copies; tasq_linear_create synchronises it before
+ *                 returning, so the caller may free its weight copies afterwards.
+ * Requires the current device to be sm_100 (B200). Allocates device memory with cudaMalloc.
+ */
+tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, int32_t num_layers,
+                               int32_t num_steps, int32_t hadamard_n, int64_t max_tokens,
+                               int32_t out_dtype, void* stream);
+
+/*
+ * Replace the schedule table with bits_host [num_layers * num_steps] (host, row-major by layer,
+ * every entry in [1, 8]; bits = 8 keeps all bit planes, bits = b keeps the top b planes).
+ * Stream-ordered: forwards enqueued on `stream` after this call see the new table. The host
+ * array may be reused as soon as the call returns. No kernel is launched and the weight
+ * buffer is never touched: the table is the only thing that changes between steps.
+ */
+tasq_status tasq_set_schedule(tasq_ctx* ctx, const uint8_t* bits_host, void* stream);
+
+/*
+ * y = dequant( Q(x H) . mask(W_layer, bits[layer][step])^T )  for one layer at one step.
+ *   x     : device FP16 activations [M, K_layer], row stride ldx (elements, >= K, % 8 == 0).
+ *   M     : tokens, 0 <= M <= max_tokens (M == 0 enqueues nothing).
+ *   layer : 0 <= layer < num_layers.   step : 0 <= step < num_steps.
+ *   y     : device outputs [M, N_layer] in the context's out_dtype, row stride ldy
+ *           (elements, >= N, % 8 == 0).
+ * Two kernels run on `stream`: the prologue (block Hadamard of size n along K with zero
+ * padding to Kp, per-token absmax, s_x = absmax / (127 sqrt(n)), codes RNE(z * 127 / absmax)
+ * in [-127, 127]) into the context workspace, then the GEMM, which reads bits[layer][step]
+ * from the device table, clears the low bit planes of each weight tile as it streams into
+ * shared memory, accumulates exactly in INT32 and writes y = acc * s_x[m] * s_w[n].
+ * Uses the context workspace: forwards of one context must not overlap in time on different
+ * streams.
+ */
+tasq_status tasq_linear_forward(tasq_ctx* ctx, const void* x, int64_t M, int64_t ldx, int32_t layer,
+                                int32_t step, void* y, int64_t ldy, void* stream);
+
+/* Free every device allocation of the context (synchronises the device first). NULL is a no-op. */
+tasq_status tasq_linear_destroy(tasq_ctx* ctx);
+
+/* Message of the last failing call on this thread ("" if none). Valid until the next call. */
+const char* tasq_last_error(void);
+
+/*
+ * Read the context's device status word (0 = healthy; otherwise TASQ_DEVICE_* bits of bounded
+ * waits that ran out or of invalid table entries). Synchronises `stream`. If `clear` is
+ * non-zero the word is reset to 0 afterwards.
+ */
+tasq_status tasq_get_device_status(tasq_ctx* ctx, uint32_t* status_out, int32_t clear, void* stream);
+
+/*
+ * Bound for every device-side wait of the context's kernels, in nanoseconds (default 1e9).
+ * A wait that runs out sets a status bit and makes its kernel wind down and return.
+ */
+tasq_status tasq_set_wait_limit(tasq_ctx* ctx, uint64_t limit_ns);
+
+/* Hadamard block size, padded K and N of a layer (host queries, no device work). */
+tasq_status tasq_layer_info(const tasq_ctx* ctx, int32_t layer, int32_t* N, int32_t* K, int32_t* Kp);
+
+/*
+ * Test hooks: the same kernels as tasq_linear_forward, with caller-owned buffers.
+ *
+ * tasq_debug_quantize: prologue only. x as in tasq_linear_forward (layer selects K); writes
+ *   xq [M, Kp] INT8 (device, row stride Kp) and s_x [M] FP32 (device).
+ *
+ * tasq_debug_gemm_s32: GEMM only, raw INT32 accumulators. xq [M, Kp] INT8 (device, stride Kp);
+ *   acc [M, N] INT32 (device, row stride ld_acc >= N, % 8 == 0).
+ *
+ * tasq_debug_gemm: GEMM only with the dequantizing epilogue. xq as above, s_x [M] FP32
+ *   (device), y [M, N] in out_dtype (a tasq_out_dtype, independent of the context's).
+ */
+tasq_status tasq_debug_quantize(tasq_ctx* ctx, const void* x, int64_t M, int64_t ldx, int32_t layer,
+                                int8_t* xq, float* s_x, void* stream);
+tasq_status tasq_debug_gemm_s32(tasq_ctx* ctx, const int8_t* xq, int64_t M, int32_t layer, int32_t step,
+                                int32_t* acc, int64_t ld_acc, void* stream);
+tasq_status tasq_debug_gemm(tasq_ctx* ctx, const int8_t* xq, const float* s_x, int64_t M, int32_t layer,
+                            int32_t step, void* y, int64_t ldy, int32_t out_dtype, void* stream);
+
+/*
+ * Failure-detection hook: launch one CTA that waits, with the context's wait limit, on a
+ * shared-memory barrier that nothing ever arrives on. The wait must run out, set
+ * TASQ_DEVICE_TIMEOUT_MMA in the status word and return. Used by tests to check that a
+ * stuck wait ends with a status the host can read and leaves the context usable.
+ */
+tasq_status tasq_debug_stuck_wait(tasq_ctx* ctx, void* stream);
+
+/*
+ * Kernel timing trace (native instrumentation). When enabled with capacity > 0, every forward
+ * records CUDA events around its prologue and GEMM kernels on the forward's stream, for up to
+ * `capacity` forwards (later forwards are not recorded). tasq_trace_read synchronises the
+ * recorded events and returns, per kernel kind, the number of launches and the summed
+ * duration in milliseconds, then clears the trace. capacity 0 disables tracing.
+ */
+tasq_status tasq_trace_enable(tasq_ctx* ctx, int32_t capacity);
+tasq_status tasq_trace_read(tasq_ctx* ctx, int32_t* prologue_launches, double* prologue_ms,
+                            int32_t* gemm_launches, double* gemm_ms, double* gemm_ops, double* prologue_bytes);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TASQ_H_ */

@@ -1,0 +1,95 @@
+"""The C-ABI library loads, exports every symbol include/tasq.h declares, and rejects bad
+arguments on the host before touching a device (no compute calls: runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tasq.h")
+
+
+@pytest.fixture(scope="module")
+def tasq():
+    from timestep_adaptive_bit_b200 import build
+    build.build()
+    import timestep_adaptive_bit_b200 as t
+    return t
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tasq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("tasq_linear_create", "tasq_linear_forward", "tasq_set_schedule", "tasq_linear_destroy"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(tasq):
+    lib = ctypes.CDLL(tasq.LIB_PATH)
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, f"declared but not exported: {missing}"
+
+
+def test_binding_names_match_header(tasq):
+    for n in _declared_functions():
+        assert hasattr(tasq, n), f"binding lacks {n}"
+
+
+def test_enum_and_limits_match_header(tasq):
+    src = open(HEADER).read()
+    for name in ("TASQ_OK", "TASQ_ERR_INVALID_ARG", "TASQ_ERR_CUDA", "TASQ_ERR_UNSUPPORTED_ARCH",
+                 "TASQ_ERR_WORKSPACE", "TASQ_ERR_TIMEOUT", "TASQ_OUT_F16", "TASQ_OUT_BF16"):
+        m = re.search(rf"\b{name}\s*=\s*(\d+)", src)
+        assert m and int(m.group(1)) == getattr(tasq, name), name
+    for name in ("TASQ_DEVICE_TIMEOUT_PRODUCER", "TASQ_DEVICE_TIMEOUT_MMA", "TASQ_DEVICE_TIMEOUT_MASK",
+                 "TASQ_DEVICE_TIMEOUT_EPILOGUE", "TASQ_DEVICE_TIMEOUT_DRAIN", "TASQ_DEVICE_BAD_BITS", "TASQ_MAX_KP"):
+        m = re.search(rf"#define\s+{name}\s+(0x[0-9a-fA-F]+|\d+)u?", src)
+        assert m and int(m.group(1), 0) == getattr(tasq, name), name
+
+
+def test_layer_desc_layout(tasq):
+    d = tasq.tasq_layer_desc
+    assert ctypes.sizeof(d) == 24
+    assert d.N.offset == 0 and d.K.offset == 4 and d.w.offset == 8 and d.s_w.offset == 16
+
+
+def test_host_validation_without_device(tasq):
+    lib = tasq.lib
+    h = ctypes.c_void_p()
+    w = np.zeros((64, 64), np.int8)
+    sw = np.ones(64, np.float32)
+    desc = (tasq.tasq_layer_desc * 1)(tasq.tasq_layer_desc(64, 64, w.ctypes.data, sw.ctypes.data))
+    # bad Hadamard size, bad token count, no layers, bad dtype: all rejected before any CUDA call
+    assert lib.tasq_linear_create(ctypes.byref(h), desc, 1, 4, 32, 256, 0, None) == tasq.TASQ_ERR_INVALID_ARG
+    assert "hadamard_n" in tasq.tasq_last_error()
+    assert lib.tasq_linear_create(ctypes.byref(h), desc, 1, 4, 64, 0, 0, None) == tasq.TASQ_ERR_INVALID_ARG
+    assert lib.tasq_linear_create(ctypes.byref(h), desc, 0, 4, 64, 256, 0, None) == tasq.TASQ_ERR_INVALID_ARG
+    assert lib.tasq_linear_create(ctypes.byref(h), desc, 1, 0, 64, 256, 0, None) == tasq.TASQ_ERR_INVALID_ARG
+    assert lib.tasq_linear_create(ctypes.byref(h), desc, 1, 4, 64, 256, 7, None) == tasq.TASQ_ERR_INVALID_ARG
+    assert lib.tasq_linear_create(None, desc, 1, 4, 64, 256, 0, None) == tasq.TASQ_ERR_INVALID_ARG
+    assert h.value is None
+    # NULL contexts
+    assert lib.tasq_linear_forward(None, None, 1, 64, 0, 0, None, 64, None) == tasq.TASQ_ERR_INVALID_ARG
+    assert lib.tasq_set_schedule(None, None, None) == tasq.TASQ_ERR_INVALID_ARG
+    assert lib.tasq_set_wait_limit(None, 10 ** 9) == tasq.TASQ_ERR_INVALID_ARG
+    assert lib.tasq_linear_destroy(None) == tasq.TASQ_OK
+    with pytest.raises(tasq.TasqError) as ei:
+        tasq.tasq_linear_create([(64, 64, w, sw)], 4, 48, 256)
+    assert ei.value.status == tasq.TASQ_ERR_INVALID_ARG
+
+
+def test_no_cpu_fallback_in_product_path():
+    """The package never imports the oracle or any CPU implementation of the path."""
+    pkg = os.path.join(ROOT, "timestep_adaptive_bit_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle\b", src, flags=re.M), f

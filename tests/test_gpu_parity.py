@@ -1,0 +1,325 @@
+"""CUDA path against the CPU oracle, element by element, through the C ABI.
+
+Bars (from the method's stated tolerances):
+  * INT32 accumulators: bit-exact.
+  * INT8 activation codes: at most 0.1 % differ, none by more than 1 (both sides decide them in
+    FP32 with the same butterfly order, so they are expected to agree exactly).
+  * s_x: relative error <= 1e-6 (FP32 scale against the FP64 definition).
+  * FP16 outputs given identical codes: |dy| <= 1e-3 |y| + 2^-24 elementwise;
+    BF16 outputs: |dy| <= 2^-8 |y| + 2^-24 (one BF16 rounding of an FP32 product).
+  * Whole forward: ||dy||_F / ||y||_F <= 1e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+
+torch = pytest.importorskip("torch")
+
+pytestmark = pytest.mark.gpu
+
+F16_REL = 1e-3
+ABS_TINY = 2.0 ** -24
+
+
+@pytest.fixture(scope="module")
+def T():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from timestep_adaptive_bit_b200 import build
+    build.build()
+    import timestep_adaptive_bit_b200 as t
+    torch.cuda.init()
+    return t
+
+
+def _stream():
+    return torch.cuda.current_stream()
+
+
+def _acts(rng, M, K, outliers=True):
+    x = rng.standard_normal((M, K), dtype=np.float32)
+    if outliers:
+        cols = rng.choice(K, size=max(1, K // 200), replace=False)
+        x[:, cols] *= 50
+    return x.astype(np.float16)
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _codes_ok(q_gpu, q_ref):
+    d = np.abs(q_gpu.astype(np.int64) - q_ref.astype(np.int64))
+    assert d.max(initial=0) <= 1, f"a code differs by {d.max()}"
+    frac = d.astype(bool).mean() if d.size else 0.0
+    assert frac <= 1e-3, f"{frac:.2e} of codes differ"
+    return frac
+
+
+def _ctx(T, layers, steps, n, max_tokens, out=0):
+    return T.tasq_linear_create(layers, steps, n, max_tokens, out, _stream())
+
+
+# ----------------------------------------------------------------------------- prologue
+@pytest.mark.parametrize("n,K,M", [(64, 64, 1), (64, 96, 3), (64, 1152, 257), (128, 2240, 130), (128, 128, 5),
+                                   (64, 12288, 33), (128, 16384, 2), (64, 4608, 300), (128, 5600, 64)])
+def test_prologue_matches_oracle(T, n, K, M):
+    rng = np.random.default_rng(K * 31 + M)
+    x = _acts(rng, M, K)
+    if M >= 3:
+        x[1] = 0                    # all-zero token: codes 0, scale 0
+        x[2] = np.float16(0.5)      # constant token
+    Kp = oracle.padded_k(K, n)
+    ctx = _ctx(T, [(64, K, np.zeros((64, Kp), np.int8), np.ones(64, np.float32))], 1, n, max(M, 1))
+    ldx = K + 8                     # strided rows
+    xs = np.zeros((M, ldx), np.float16)
+    xs[:, :K] = x
+    xd = _dev(xs)
+    xq = torch.empty((M, Kp), dtype=torch.int8, device="cuda")
+    sx = torch.empty((M,), dtype=torch.float32, device="cuda")
+    T.tasq_debug_quantize(ctx, xd, M, ldx, 0, xq, sx, _stream())
+    torch.cuda.synchronize()
+    q_ref, sx_ref, _ = oracle.prologue(x, n)
+    frac = _codes_ok(xq.cpu().numpy(), q_ref)
+    assert frac == 0.0, "codes are decided in FP32 in the same butterfly order on both sides"
+    sx_g = sx.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(sx_g - sx_ref) <= 1e-6 * np.abs(sx_ref)), "s_x"
+    if M >= 3:
+        assert sx_g[1] == 0.0 and not xq[1].any().item()
+    assert T.tasq_get_device_status(ctx) == 0
+
+
+# ----------------------------------------------------------------------------- GEMM, exact
+@pytest.mark.parametrize("M,N,K,n", [(1, 1, 64, 64), (256, 128, 128, 64), (300, 200, 1152, 64), (513, 384, 192, 64),
+                                     (100, 1152, 2240, 128), (257, 130, 4608, 64), (64, 2000, 64, 64)])
+def test_gemm_s32_bit_exact_all_bits(T, M, N, K, n):
+    rng = np.random.default_rng(M * 7 + N * 13 + K)
+    Kp = oracle.padded_k(K, n)
+    w = rng.integers(-128, 128, size=(N, Kp)).astype(np.int8)     # includes -128
+    q = rng.integers(-127, 128, size=(M, Kp)).astype(np.int8)
+    steps = 8
+    ctx = _ctx(T, [(N, K, w, np.ones(N, np.float32))], steps, n, M)
+    bits = np.array([[8, 7, 6, 5, 4, 3, 2, 1]], np.uint8)
+    T.tasq_set_schedule(ctx, bits, _stream())
+    qd = _dev(q)
+    ld = N + (8 - N % 8) % 8 + 8
+    for step in range(steps):
+        acc = torch.full((M, ld), 0x7F7F7F7F, dtype=torch.int32, device="cuda")
+        T.tasq_debug_gemm_s32(ctx, qd, M, 0, step, acc, ld, _stream())
+        torch.cuda.synchronize()
+        got = acc.cpu().numpy()
+        ref = oracle.int_gemm(q, oracle.lsb_mask(w, int(bits[0, step])))
+        assert np.array_equal(got[:, :N].astype(np.int64), ref), f"INT32 accumulators differ at bits={bits[0, step]}"
+        assert np.all(got[:, N:] == 0x7F7F7F7F), "write outside [M, N]"
+    assert T.tasq_get_device_status(ctx) == 0
+
+
+def test_gemm_extreme_values(T):
+    """All-(-128) weights at k = 0 and all-(-127) codes: the largest accumulators at Kp = 12288."""
+    M, N, K = 256, 128, 12288
+    w = np.full((N, K), -128, np.int8)
+    w[::2] = 127
+    q = np.full((M, K), -127, np.int8)
+    q[::3] = 127
+    ctx = _ctx(T, [(N, K, w, np.ones(N, np.float32))], 2, 64, M)
+    T.tasq_set_schedule(ctx, np.array([[8, 1]], np.uint8), _stream())
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    for step, bits in ((0, 8), (1, 1)):
+        T.tasq_debug_gemm_s32(ctx, _dev(q), M, 0, step, acc, N, _stream())
+        torch.cuda.synchronize()
+        ref = oracle.int_gemm(q, oracle.lsb_mask(w, bits))
+        assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref)
+
+
+# ----------------------------------------------------------------------------- dequant epilogue
+@pytest.mark.parametrize("out", [0, 1])
+@pytest.mark.parametrize("M,N,K", [(300, 200, 1152), (17, 1152, 64), (512, 256, 256)])
+def test_gemm_dequant_given_codes(T, out, M, N, K):
+    rng = np.random.default_rng(M + N + K + out)
+    w = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+    q = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+    s_x = rng.uniform(0.01, 3.0, size=M).astype(np.float32)
+    s_x[0] = 0.0
+    ctx = _ctx(T, [(N, K, w, s_w)], 2, 64, M)
+    T.tasq_set_schedule(ctx, np.array([[8, 5]], np.uint8), _stream())
+    tdt = torch.float16 if out == 0 else torch.bfloat16
+    for step, bits in ((0, 8), (1, 5)):
+        y = torch.full((M, N), float("nan"), dtype=tdt, device="cuda")
+        T.tasq_debug_gemm(ctx, _dev(q), _dev(s_x), M, 0, step, y, N, out, _stream())
+        torch.cuda.synchronize()
+        got = y.float().cpu().numpy().astype(np.float64)
+        ref = oracle.dequant(oracle.int_gemm(q, oracle.lsb_mask(w, bits)), s_x, s_w)
+        rel = F16_REL if out == 0 else 2.0 ** -8
+        assert np.all(np.abs(got - ref) <= rel * np.abs(ref) + ABS_TINY), "dequantized outputs"
+
+
+# ----------------------------------------------------------------------------- whole forward
+@pytest.mark.parametrize("n,K,N,M", [(64, 1152, 1152, 256), (64, 1152, 3456, 300), (128, 2240, 6720, 130),
+                                     (64, 4608, 1152, 77), (128, 5600, 2240, 513), (64, 64, 8, 1)])
+def test_forward_matches_oracle(T, n, K, N, M):
+    rng = np.random.default_rng(n + K + N + M)
+    Kp = oracle.padded_k(K, n)
+    x = _acts(rng, M, K)
+    w = rng.integers(-127, 128, size=(N, Kp)).astype(np.int8)
+    s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+    bits_per_step = [8, 6, 5, 4, 3]
+    ctx = _ctx(T, [(N, K, w, s_w)], len(bits_per_step), n, M + 5)
+    T.tasq_set_schedule(ctx, np.array([bits_per_step], np.uint8), _stream())
+    xd = _dev(x)
+    ldy = N + (8 - N % 8) % 8 + 16
+    ref_q, ref_sx, _ = oracle.prologue(x, n)
+    for step, bits in enumerate(bits_per_step):
+        y = torch.full((M + 2, ldy), float("nan"), dtype=torch.float16, device="cuda")
+        T.tasq_linear_forward(ctx, xd, M, K, 0, step, y, ldy, _stream())
+        torch.cuda.synchronize()
+        got_all = y.float().cpu().numpy()
+        assert np.isnan(got_all[:M, N:]).all() and np.isnan(got_all[M:]).all(), "write outside [M, N]"
+        got = got_all[:M, :N].astype(np.float64)
+        ref = oracle.masked_linear(x, w, s_w, bits, n)["y"]
+        assert np.linalg.norm(got - ref) <= 1e-3 * np.linalg.norm(ref)
+        assert np.all(np.abs(got - ref) <= F16_REL * np.abs(ref) + ABS_TINY), "elementwise (codes agree exactly)"
+    assert T.tasq_get_device_status(ctx) == 0
+
+
+def test_schedule_is_stream_ordered(T):
+    """A schedule change between two forwards on one stream affects only the later forward, and
+    the weights are never rewritten (the same buffer serves both)."""
+    rng = np.random.default_rng(3)
+    M, K, N, n = 256, 1152, 1152, 64
+    x = _acts(rng, M, K)
+    w = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+    ctx = _ctx(T, [(N, K, w, s_w)], 1, n, M)
+    xd = _dev(x)
+    ys = [torch.empty((M, N), dtype=torch.float16, device="cuda") for _ in range(3)]
+    s = _stream()
+    T.tasq_set_schedule(ctx, np.array([[8]], np.uint8), s)
+    T.tasq_linear_forward(ctx, xd, M, K, 0, 0, ys[0], N, s)
+    T.tasq_set_schedule(ctx, np.array([[3]], np.uint8), s)
+    T.tasq_linear_forward(ctx, xd, M, K, 0, 0, ys[1], N, s)
+    T.tasq_set_schedule(ctx, np.array([[8]], np.uint8), s)
+    T.tasq_linear_forward(ctx, xd, M, K, 0, 0, ys[2], N, s)
+    torch.cuda.synchronize()
+    for y, bits in zip(ys, (8, 3, 8)):
+        ref = oracle.masked_linear(x, w, s_w, bits, n)["y"]
+        got = y.float().cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(got - ref) <= F16_REL * np.abs(ref) + ABS_TINY)
+    assert torch.equal(ys[0], ys[2])
+
+
+def test_multi_layer_context_uses_each_layers_weights(T):
+    rng = np.random.default_rng(9)
+    n, M = 64, 200
+    shapes = [(1152, 3456), (1152, 1152), (4608, 1152), (64, 200)]
+    layers, xs = [], []
+    for K, N in shapes:
+        w = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+        s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+        layers.append((N, K, w, s_w))
+        xs.append(_acts(rng, M, K))
+    ctx = _ctx(T, layers, 3, n, M)
+    sched = np.array([[8, 4, 6], [5, 8, 2], [7, 7, 1], [1, 2, 3]], np.uint8)
+    T.tasq_set_schedule(ctx, sched, _stream())
+    for layer, ((N, K, w, s_w), x) in enumerate(zip(layers, xs)):
+        for step in range(3):
+            assert T.tasq_layer_info(ctx, layer) == (N, K, K)
+            y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+            T.tasq_linear_forward(ctx, _dev(x), M, K, layer, step, y, N, _stream())
+            torch.cuda.synchronize()
+            ref = oracle.masked_linear(x, w, s_w, int(sched[layer, step]), n)["y"]
+            got = y.float().cpu().numpy().astype(np.float64)
+            assert np.all(np.abs(got - ref) <= F16_REL * np.abs(ref) + ABS_TINY), (layer, step)
+
+
+def test_bf16_forward(T):
+    rng = np.random.default_rng(21)
+    M, K, N, n = 130, 2240, 700, 128
+    Kp = oracle.padded_k(K, n)
+    x = _acts(rng, M, K)
+    w = rng.integers(-127, 128, size=(N, Kp)).astype(np.int8)
+    s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+    ctx = _ctx(T, [(N, K, w, s_w)], 1, n, M, out=1)
+    T.tasq_set_schedule(ctx, np.array([[6]], np.uint8), _stream())
+    ldy = 704                       # N = 700 is ragged; the row stride must be a multiple of 8
+    y = torch.empty((M, ldy), dtype=torch.bfloat16, device="cuda")
+    T.tasq_linear_forward(ctx, _dev(x), M, K, 0, 0, y, ldy, _stream())
+    torch.cuda.synchronize()
+    ref = oracle.masked_linear(x, w, s_w, 6, n)["y"]
+    got = y[:, :N].float().cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + ABS_TINY)
+
+
+# ----------------------------------------------------------------------------- errors and status
+def test_argument_errors_on_device(T):
+    rng = np.random.default_rng(1)
+    M, K, N = 64, 128, 64
+    w = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    ctx = _ctx(T, [(N, K, w, np.ones(N, np.float32))], 2, 64, M)
+    x = torch.zeros((M + 1, K), dtype=torch.float16, device="cuda")
+    y = torch.zeros((M + 1, N + 8), dtype=torch.float16, device="cuda")
+    s = _stream()
+
+    def err(fn, *a):
+        with pytest.raises(T.TasqError) as ei:
+            fn(*a)
+        return ei.value.status
+
+    assert err(T.tasq_linear_forward, ctx, x, M + 1, K, 0, 0, y, N, s) == T.TASQ_ERR_WORKSPACE
+    assert err(T.tasq_linear_forward, ctx, x.data_ptr() + 2, M, K, 0, 0, y, N, s) == T.TASQ_ERR_INVALID_ARG
+    assert err(T.tasq_linear_forward, ctx, x, M, K - 4, 0, 0, y, N, s) == T.TASQ_ERR_INVALID_ARG
+    assert err(T.tasq_linear_forward, ctx, x, M, K, 1, 0, y, N, s) == T.TASQ_ERR_INVALID_ARG
+    assert err(T.tasq_linear_forward, ctx, x, M, K, 0, 2, y, N, s) == T.TASQ_ERR_INVALID_ARG
+    assert err(T.tasq_linear_forward, ctx, x, M, K, 0, -1, y, N, s) == T.TASQ_ERR_INVALID_ARG
+    assert err(T.tasq_linear_forward, ctx, x, M, K, 0, 0, y, N + 3, s) == T.TASQ_ERR_INVALID_ARG
+    assert err(T.tasq_linear_forward, ctx, x, -1, K, 0, 0, y, N, s) == T.TASQ_ERR_INVALID_ARG
+    assert err(T.tasq_set_schedule, ctx, np.array([[8, 0]], np.uint8), s) == T.TASQ_ERR_INVALID_ARG
+    assert err(T.tasq_set_schedule, ctx, np.array([[9, 8]], np.uint8), s) == T.TASQ_ERR_INVALID_ARG
+    T.tasq_linear_forward(ctx, x, 0, K, 0, 0, y, N, s)        # M = 0: nothing to do
+    assert T.tasq_get_device_status(ctx) == 0
+    with pytest.raises(T.TasqError):
+        T.tasq_linear_create([(N, 12, w, np.ones(N, np.float32))], 1, 64, 8)   # K % 8 != 0
+    with pytest.raises(T.TasqError):
+        T.tasq_linear_create([(N, 16392, np.zeros((N, 16448), np.int8), np.ones(N, np.float32))], 1, 64, 8)
+
+
+def test_stuck_wait_times_out_and_context_stays_usable(T):
+    """A wait on a barrier nothing arrives on runs out, reports a status bit, and the context
+    keeps working afterwards (failure detected on the host, no fault, no trap)."""
+    rng = np.random.default_rng(5)
+    M, K, N, n = 256, 1152, 256, 64
+    x = _acts(rng, M, K)
+    w = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+    ctx = _ctx(T, [(N, K, w, s_w)], 1, n, M)
+    T.tasq_set_wait_limit(ctx, 20_000_000)       # 20 ms
+    T.tasq_debug_stuck_wait(ctx, _stream())
+    st = T.tasq_get_device_status(ctx, clear=True)
+    assert st & T.TASQ_DEVICE_TIMEOUT_MMA
+    assert T.tasq_get_device_status(ctx) == 0
+    T.tasq_set_wait_limit(ctx, 1_000_000_000)
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    T.tasq_linear_forward(ctx, _dev(x), M, K, 0, 0, y, N, _stream())
+    torch.cuda.synchronize()
+    ref = oracle.masked_linear(x, w, s_w, 8, n)["y"]
+    assert np.all(np.abs(y.float().cpu().numpy() - ref) <= F16_REL * np.abs(ref) + ABS_TINY)
+    assert T.tasq_get_device_status(ctx) == 0
+
+
+def test_trace_counts_launches(T):
+    rng = np.random.default_rng(8)
+    M, K, N = 256, 1152, 1152
+    w = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    ctx = _ctx(T, [(N, K, w, np.ones(N, np.float32))], 1, 64, M)
+    T.tasq_trace_enable(ctx, 4)
+    x = _dev(_acts(rng, M, K))
+    y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    for _ in range(6):
+        T.tasq_linear_forward(ctx, x, M, K, 0, 0, y, N, _stream())
+    tr = T.tasq_trace_read(ctx)
+    assert tr["gemm_launches"] == 4 and tr["prologue_launches"] == 4
+    assert tr["gemm_ms"] > 0 and tr["prologue_ms"] > 0
+    assert tr["gemm_ops"] == 4 * 2.0 * M * N * K

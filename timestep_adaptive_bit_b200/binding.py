@@ -1,0 +1,222 @@
+"""ctypes binding of libtasq (include/tasq.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls. Tensors may be passed as
+torch tensors (their data_ptr() is used) or as raw integer addresses; streams as a
+torch.cuda.Stream, a raw cudaStream_t integer, or None (the legacy default stream). A non-zero
+status raises TasqError carrying tasq_last_error(). There is no fallback: if libtasq.so is
+missing the import fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Iterable, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtasq.so")
+
+TASQ_OK = 0
+TASQ_ERR_INVALID_ARG = 1
+TASQ_ERR_CUDA = 2
+TASQ_ERR_UNSUPPORTED_ARCH = 3
+TASQ_ERR_WORKSPACE = 4
+TASQ_ERR_TIMEOUT = 5
+
+TASQ_OUT_F16 = 0
+TASQ_OUT_BF16 = 1
+
+TASQ_DEVICE_TIMEOUT_PRODUCER = 0x1
+TASQ_DEVICE_TIMEOUT_MMA = 0x2
+TASQ_DEVICE_TIMEOUT_MASK = 0x4
+TASQ_DEVICE_TIMEOUT_EPILOGUE = 0x8
+TASQ_DEVICE_TIMEOUT_DRAIN = 0x10
+TASQ_DEVICE_BAD_BITS = 0x100
+
+TASQ_MAX_KP = 16384
+
+
+class TasqError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"tasq status {status}: {message}")
+        self.status = status
+        self.message = message
+
+
+class tasq_layer_desc(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("w", ctypes.c_void_p), ("s_w", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m timestep_adaptive_bit_b200.build` "
+            "(or __graft_entry__.build()); there is no fallback implementation")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    i32, i64, u64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64
+    sigs = {
+        "tasq_linear_create": [ctypes.POINTER(P), ctypes.POINTER(tasq_layer_desc), i32, i32, i32, i64, i32, P],
+        "tasq_set_schedule": [P, P, P],
+        "tasq_linear_forward": [P, P, i64, i64, i32, i32, P, i64, P],
+        "tasq_linear_destroy": [P],
+        "tasq_get_device_status": [P, ctypes.POINTER(ctypes.c_uint32), i32, P],
+        "tasq_set_wait_limit": [P, u64],
+        "tasq_layer_info": [P, i32, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)],
+        "tasq_debug_quantize": [P, P, i64, i64, i32, P, P, P],
+        "tasq_debug_gemm_s32": [P, P, i64, i32, i32, P, i64, P],
+        "tasq_debug_gemm": [P, P, P, i64, i32, i32, P, i64, i32, P],
+        "tasq_debug_stuck_wait": [P, P],
+        "tasq_trace_enable": [P, i32],
+        "tasq_trace_read": [P, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i32),
+                            ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
+                            ctypes.POINTER(ctypes.c_double)],
+    }
+    for name, args in sigs.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    lib.tasq_last_error.argtypes = []
+    lib.tasq_last_error.restype = ctypes.c_char_p
+    return lib
+
+
+lib = _load()
+
+
+def tasq_last_error() -> str:
+    return lib.tasq_last_error().decode(errors="replace")
+
+
+def _check(status: int) -> None:
+    if status != TASQ_OK:
+        raise TasqError(status, tasq_last_error())
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if hasattr(t, "data_ptr"):
+        return int(t.data_ptr())
+    if isinstance(t, np.ndarray):
+        return int(t.ctypes.data)
+    raise TypeError(f"cannot take the address of {type(t)}")
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    if hasattr(s, "cuda_stream"):
+        return int(s.cuda_stream)
+    raise TypeError(f"not a stream: {type(s)}")
+
+
+class Context:
+    """Opaque tasq_ctx* handle (frees itself when garbage-collected if not destroyed)."""
+
+    def __init__(self, handle: int, layers: Sequence[tuple]):
+        self.handle = handle
+        self.layers = [(int(N), int(K)) for N, K, *_ in layers]
+
+    @property
+    def _as_parameter_(self):
+        return ctypes.c_void_p(self.handle)
+
+    def __del__(self):
+        if getattr(self, "handle", None):
+            try:
+                lib.tasq_linear_destroy(ctypes.c_void_p(self.handle))
+            except Exception:
+                pass
+            self.handle = None
+
+
+def tasq_linear_create(layers: Iterable[tuple], num_steps: int, hadamard_n: int, max_tokens: int,
+                       out_dtype: int = TASQ_OUT_F16, stream=None) -> Context:
+    """layers: iterable of (N, K, w, s_w) with w [N, Kp] int8 and s_w [N] float32 (host numpy
+    arrays or device tensors)."""
+    layers = list(layers)
+    arr = (tasq_layer_desc * len(layers))()
+    keep = []
+    for i, (N, K, w, s_w) in enumerate(layers):
+        if isinstance(w, np.ndarray):
+            w = np.ascontiguousarray(w, dtype=np.int8)
+            keep.append(w)
+        if isinstance(s_w, np.ndarray):
+            s_w = np.ascontiguousarray(s_w, dtype=np.float32)
+            keep.append(s_w)
+        arr[i] = tasq_layer_desc(int(N), int(K), _ptr(w), _ptr(s_w))
+    h = ctypes.c_void_p()
+    _check(lib.tasq_linear_create(ctypes.byref(h), arr, len(layers), int(num_steps), int(hadamard_n),
+                                  int(max_tokens), int(out_dtype), _stream(stream)))
+    del keep
+    return Context(h.value, layers)
+
+
+def tasq_set_schedule(ctx: Context, bits, stream=None) -> None:
+    b = np.ascontiguousarray(bits, dtype=np.uint8)
+    _check(lib.tasq_set_schedule(ctx, b.ctypes.data, _stream(stream)))
+
+
+def tasq_linear_forward(ctx: Context, x, M: int, ldx: int, layer: int, step: int, y, ldy: int, stream=None) -> None:
+    _check(lib.tasq_linear_forward(ctx, _ptr(x), int(M), int(ldx), int(layer), int(step), _ptr(y), int(ldy),
+                                   _stream(stream)))
+
+
+def tasq_linear_destroy(ctx: Context) -> None:
+    if ctx.handle:
+        h, ctx.handle = ctx.handle, None
+        _check(lib.tasq_linear_destroy(ctypes.c_void_p(h)))
+
+
+def tasq_get_device_status(ctx: Context, clear: bool = False, stream=None) -> int:
+    v = ctypes.c_uint32(0)
+    _check(lib.tasq_get_device_status(ctx, ctypes.byref(v), 1 if clear else 0, _stream(stream)))
+    return int(v.value)
+
+
+def tasq_set_wait_limit(ctx: Context, limit_ns: int) -> None:
+    _check(lib.tasq_set_wait_limit(ctx, int(limit_ns)))
+
+
+def tasq_layer_info(ctx: Context, layer: int):
+    N, K, Kp = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(lib.tasq_layer_info(ctx, int(layer), ctypes.byref(N), ctypes.byref(K), ctypes.byref(Kp)))
+    return int(N.value), int(K.value), int(Kp.value)
+
+
+def tasq_debug_quantize(ctx: Context, x, M: int, ldx: int, layer: int, xq, s_x, stream=None) -> None:
+    _check(lib.tasq_debug_quantize(ctx, _ptr(x), int(M), int(ldx), int(layer), _ptr(xq), _ptr(s_x), _stream(stream)))
+
+
+def tasq_debug_gemm_s32(ctx: Context, xq, M: int, layer: int, step: int, acc, ld_acc: int, stream=None) -> None:
+    _check(lib.tasq_debug_gemm_s32(ctx, _ptr(xq), int(M), int(layer), int(step), _ptr(acc), int(ld_acc),
+                                   _stream(stream)))
+
+
+def tasq_debug_gemm(ctx: Context, xq, s_x, M: int, layer: int, step: int, y, ldy: int, out_dtype: int,
+                    stream=None) -> None:
+    _check(lib.tasq_debug_gemm(ctx, _ptr(xq), _ptr(s_x), int(M), int(layer), int(step), _ptr(y), int(ldy),
+                               int(out_dtype), _stream(stream)))
+
+
+def tasq_debug_stuck_wait(ctx: Context, stream=None) -> None:
+    _check(lib.tasq_debug_stuck_wait(ctx, _stream(stream)))
+
+
+def tasq_trace_enable(ctx: Context, capacity: int) -> None:
+    _check(lib.tasq_trace_enable(ctx, int(capacity)))
+
+
+def tasq_trace_read(ctx: Context) -> dict:
+    pl, gl = ctypes.c_int32(), ctypes.c_int32()
+    pm, gm, ops, pb = ctypes.c_double(), ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+    _check(lib.tasq_trace_read(ctx, ctypes.byref(pl), ctypes.byref(pm), ctypes.byref(gl), ctypes.byref(gm),
+                               ctypes.byref(ops), ctypes.byref(pb)))
+    return {"prologue_launches": pl.value, "prologue_ms": pm.value, "gemm_launches": gl.value,
+            "gemm_ms": gm.value, "gemm_ops": ops.value, "prologue_bytes": pb.value}

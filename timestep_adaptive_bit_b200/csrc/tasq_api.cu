@@ -1,0 +1,506 @@
+// C ABI of the masked INT8 linear: context (one shared weight buffer, device schedule table,
+// activation workspace), argument validation, TMA descriptors and kernel launches.
+#include <cudaTypedefs.h>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/tasq.h"
+#include "tasq_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+tasq_status fail(tasq_status st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+
+tasq_status fail_cuda(cudaError_t e, const char* what) {
+  std::string m = std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+  return fail(TASQ_ERR_CUDA, m);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D UINT8 tensor [rows, cols] with row stride `cols` bytes, loaded in boxes of
+// box_cols x box_rows with 128-byte swizzle; out-of-range elements read as zero.
+tasq_status make_tmap_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                         uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(TASQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TASQ_ERR_CUDA, "cuTensorMapEncodeTiled failed with CUresult " + std::to_string(r));
+  return TASQ_OK;
+}
+
+struct LayerInfo {
+  int32_t N, K, Kp;
+  size_t w_off;    // bytes into the weight buffer
+  size_t sw_off;   // floats into the scale buffer
+};
+
+struct TraceRec {
+  cudaEvent_t e0, e1, e2;
+  double ops, bytes;
+};
+
+}  // namespace
+
+struct tasq_ctx {
+  int device = -1;
+  int num_sms = 0;
+  int32_t num_layers = 0, num_steps = 0, n = 0, out_dtype = 0;
+  int64_t max_tokens = 0;
+  int32_t kp_max = 0;
+  std::vector<LayerInfo> layers;
+  std::vector<CUtensorMap> tmap_w;
+  int8_t* d_w = nullptr;
+  float* d_sw = nullptr;
+  uint8_t* d_bits = nullptr;
+  int8_t* d_xq = nullptr;
+  float* d_sx = nullptr;
+  uint32_t* d_status = nullptr;
+  uint64_t wait_limit_ns = 1000000000ull;
+  float sx_factor = 0.0f;
+  // trace
+  int32_t trace_cap = 0, trace_count = 0;
+  std::vector<TraceRec> trace;
+};
+
+namespace {
+
+void free_ctx(tasq_ctx* c) {
+  if (c == nullptr) return;
+  if (c->device >= 0) cudaSetDevice(c->device);
+  cudaDeviceSynchronize();
+  cudaFree(c->d_w);
+  cudaFree(c->d_sw);
+  cudaFree(c->d_bits);
+  cudaFree(c->d_xq);
+  cudaFree(c->d_sx);
+  cudaFree(c->d_status);
+  for (auto& t : c->trace) {
+    cudaEventDestroy(t.e0);
+    cudaEventDestroy(t.e1);
+    cudaEventDestroy(t.e2);
+  }
+  delete c;
+}
+
+tasq_status check_device(const tasq_ctx* c) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  if (dev != c->device)
+    return fail(TASQ_ERR_INVALID_ARG, "current device " + std::to_string(dev) + " is not the context's device " +
+                                          std::to_string(c->device));
+  return TASQ_OK;
+}
+
+tasq_status check_layer(const tasq_ctx* c, int32_t layer) {
+  if (layer < 0 || layer >= c->num_layers)
+    return fail(TASQ_ERR_INVALID_ARG, "layer " + std::to_string(layer) + " out of range [0, " +
+                                          std::to_string(c->num_layers) + ")");
+  return TASQ_OK;
+}
+
+tasq_status check_step(const tasq_ctx* c, int32_t step) {
+  if (step < 0 || step >= c->num_steps)
+    return fail(TASQ_ERR_INVALID_ARG,
+                "step " + std::to_string(step) + " out of range [0, " + std::to_string(c->num_steps) + ")");
+  return TASQ_OK;
+}
+
+tasq_status check_tokens(const tasq_ctx* c, int64_t M) {
+  if (M < 0) return fail(TASQ_ERR_INVALID_ARG, "M must be >= 0");
+  if (M > c->max_tokens)
+    return fail(TASQ_ERR_WORKSPACE,
+                "M = " + std::to_string(M) + " exceeds max_tokens = " + std::to_string(c->max_tokens));
+  return TASQ_OK;
+}
+
+tasq_status check_rows(const void* p, int64_t ld, int64_t width, const char* name) {
+  if (p == nullptr) return fail(TASQ_ERR_INVALID_ARG, std::string(name) + " is NULL");
+  if (!aligned16(p)) return fail(TASQ_ERR_INVALID_ARG, std::string(name) + " is not 16-byte aligned");
+  if (ld < width || ld % 8 != 0)
+    return fail(TASQ_ERR_INVALID_ARG, std::string("row stride of ") + name + " must be >= " + std::to_string(width) +
+                                          " and a multiple of 8, got " + std::to_string(ld));
+  return TASQ_OK;
+}
+
+tasq_status run_prologue(tasq_ctx* c, const LayerInfo& L, const void* x, int64_t M, int64_t ldx, int8_t* xq, float* sx,
+                         cudaStream_t s) {
+  tasq::PrologueArgs a{};
+  a.x = x;
+  a.ldx = ldx;
+  a.K = L.K;
+  a.Kp = L.Kp;
+  a.M = M;
+  a.xq = xq;
+  a.s_x = sx;
+  a.n = c->n;
+  a.sx_factor = c->sx_factor;
+  cudaError_t e = tasq::launch_prologue(a, s);
+  if (e != cudaSuccess) return fail_cuda(e, "prologue launch");
+  return TASQ_OK;
+}
+
+tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq, const float* sx, int64_t M,
+                     void* y, int64_t ldy, tasq::OutKind out, cudaStream_t s) {
+  const LayerInfo& L = c->layers[layer];
+  CUtensorMap tx;
+  tasq_status st = make_tmap_u8(&tx, xq, static_cast<uint64_t>(L.Kp), static_cast<uint64_t>(M), tasq::kGemmBlockK,
+                                tasq::kGemmTileTok);
+  if (st != TASQ_OK) return st;
+  tasq::GemmArgs g{};
+  g.M = static_cast<int32_t>(M);
+  g.N = L.N;
+  g.num_kb = (L.Kp + tasq::kGemmBlockK - 1) / tasq::kGemmBlockK;
+  g.num_m_tiles = static_cast<int32_t>((M + tasq::kGemmTileTok - 1) / tasq::kGemmTileTok);
+  g.num_n_tiles = (L.N + tasq::kGemmTileCh - 1) / tasq::kGemmTileCh;
+  g.bits_table = c->d_bits;
+  g.bits_index = layer * c->num_steps + step;
+  g.s_x = sx;
+  g.s_w = c->d_sw + L.sw_off;
+  g.y = y;
+  g.ldy = ldy;
+  g.status = c->d_status;
+  g.wait_limit_ns = c->wait_limit_ns;
+  cudaError_t e = tasq::launch_masked_gemm(c->tmap_w[layer], tx, g, out, c->num_sms, s);
+  if (e != cudaSuccess) return fail_cuda(e, "masked GEMM launch");
+  return TASQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tasq_last_error(void) { return g_last_error.c_str(); }
+
+tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, int32_t num_layers, int32_t num_steps,
+                               int32_t hadamard_n, int64_t max_tokens, int32_t out_dtype, void* stream) {
+  g_last_error.clear();
+  if (out == nullptr) return fail(TASQ_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (layers == nullptr || num_layers <= 0) return fail(TASQ_ERR_INVALID_ARG, "need at least one layer");
+  if (num_steps <= 0) return fail(TASQ_ERR_INVALID_ARG, "num_steps must be >= 1");
+  if (hadamard_n != 64 && hadamard_n != 128) return fail(TASQ_ERR_INVALID_ARG, "hadamard_n must be 64 or 128");
+  if (max_tokens <= 0 || max_tokens > 0x7fffffffLL)
+    return fail(TASQ_ERR_INVALID_ARG, "max_tokens must be in [1, 2^31 - 1]");
+  if (out_dtype != TASQ_OUT_F16 && out_dtype != TASQ_OUT_BF16)
+    return fail(TASQ_ERR_INVALID_ARG, "out_dtype must be TASQ_OUT_F16 or TASQ_OUT_BF16");
+  if (static_cast<int64_t>(num_layers) * num_steps > (1LL << 30))
+    return fail(TASQ_ERR_INVALID_ARG, "schedule table too large");
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDeviceProperties");
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(TASQ_ERR_UNSUPPORTED_ARCH, std::string("device ") + prop.name + " is sm_" + std::to_string(prop.major) +
+                                               std::to_string(prop.minor) + ", this library is built for sm_100a");
+
+  std::vector<LayerInfo> info(num_layers);
+  size_t w_bytes = 0, sw_count = 0;
+  int32_t kp_max = 0;
+  for (int32_t l = 0; l < num_layers; ++l) {
+    const tasq_layer_desc& d = layers[l];
+    if (d.N <= 0 || d.K < 8 || d.K % 8 != 0)
+      return fail(TASQ_ERR_INVALID_ARG, "layer " + std::to_string(l) + ": need N >= 1 and K >= 8 with K % 8 == 0");
+    if (d.w == nullptr || d.s_w == nullptr)
+      return fail(TASQ_ERR_INVALID_ARG, "layer " + std::to_string(l) + ": weights or scales are NULL");
+    const int32_t Kp = (d.K + hadamard_n - 1) / hadamard_n * hadamard_n;
+    if (Kp > TASQ_MAX_KP)
+      return fail(TASQ_ERR_INVALID_ARG, "layer " + std::to_string(l) + ": padded K " + std::to_string(Kp) +
+                                            " exceeds " + std::to_string(TASQ_MAX_KP));
+    info[l] = LayerInfo{d.N, d.K, Kp, w_bytes, sw_count};
+    w_bytes = round_up(w_bytes + static_cast<size_t>(d.N) * Kp, 1024);
+    sw_count = round_up(sw_count + d.N, 64);
+    if (Kp > kp_max) kp_max = Kp;
+  }
+
+  tasq_ctx* c = new tasq_ctx();
+  c->device = dev;
+  c->num_sms = prop.multiProcessorCount;
+  c->num_layers = num_layers;
+  c->num_steps = num_steps;
+  c->n = hadamard_n;
+  c->out_dtype = out_dtype;
+  c->max_tokens = max_tokens;
+  c->kp_max = kp_max;
+  c->layers = info;
+  c->sx_factor = static_cast<float>(1.0 / (127.0 * std::sqrt(static_cast<double>(hadamard_n))));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  auto bail = [&](cudaError_t err, const char* what) {
+    tasq_status st = fail_cuda(err, what);
+    free_ctx(c);
+    return st;
+  };
+  if ((e = cudaMalloc(&c->d_w, w_bytes)) != cudaSuccess) return bail(e, "cudaMalloc(weights)");
+  if ((e = cudaMalloc(&c->d_sw, sw_count * sizeof(float))) != cudaSuccess) return bail(e, "cudaMalloc(scales)");
+  const size_t table = static_cast<size_t>(num_layers) * num_steps;
+  if ((e = cudaMalloc(&c->d_bits, table)) != cudaSuccess) return bail(e, "cudaMalloc(schedule)");
+  if ((e = cudaMalloc(&c->d_xq, static_cast<size_t>(max_tokens) * kp_max)) != cudaSuccess)
+    return bail(e, "cudaMalloc(workspace codes)");
+  if ((e = cudaMalloc(&c->d_sx, static_cast<size_t>(max_tokens) * sizeof(float))) != cudaSuccess)
+    return bail(e, "cudaMalloc(workspace scales)");
+  if ((e = cudaMalloc(&c->d_status, sizeof(uint32_t))) != cudaSuccess) return bail(e, "cudaMalloc(status)");
+
+  if ((e = cudaMemsetAsync(c->d_bits, 8, table, s)) != cudaSuccess) return bail(e, "cudaMemsetAsync(schedule)");
+  if ((e = cudaMemsetAsync(c->d_status, 0, sizeof(uint32_t), s)) != cudaSuccess) return bail(e, "cudaMemsetAsync(status)");
+  for (int32_t l = 0; l < num_layers; ++l) {
+    const LayerInfo& L = info[l];
+    e = cudaMemcpyAsync(c->d_w + L.w_off, layers[l].w, static_cast<size_t>(L.N) * L.Kp, cudaMemcpyDefault, s);
+    if (e != cudaSuccess) return bail(e, "copy of weights");
+    e = cudaMemcpyAsync(c->d_sw + L.sw_off, layers[l].s_w, static_cast<size_t>(L.N) * sizeof(float),
+                        cudaMemcpyDefault, s);
+    if (e != cudaSuccess) return bail(e, "copy of weight scales");
+  }
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return bail(e, "cudaStreamSynchronize");
+
+  c->tmap_w.resize(num_layers);
+  for (int32_t l = 0; l < num_layers; ++l) {
+    const LayerInfo& L = info[l];
+    tasq_status st = make_tmap_u8(&c->tmap_w[l], c->d_w + L.w_off, static_cast<uint64_t>(L.Kp),
+                                  static_cast<uint64_t>(L.N), tasq::kGemmBlockK, tasq::kGemmTileCh);
+    if (st != TASQ_OK) {
+      std::string m = g_last_error;
+      free_ctx(c);
+      return fail(st, m);
+    }
+  }
+  *out = c;
+  return TASQ_OK;
+}
+
+tasq_status tasq_set_schedule(tasq_ctx* c, const uint8_t* bits_host, void* stream) {
+  g_last_error.clear();
+  if (c == nullptr || bits_host == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx or bits is NULL");
+  tasq_status st = check_device(c);
+  if (st != TASQ_OK) return st;
+  const size_t table = static_cast<size_t>(c->num_layers) * c->num_steps;
+  for (size_t i = 0; i < table; ++i) {
+    if (bits_host[i] < 1 || bits_host[i] > 8)
+      return fail(TASQ_ERR_INVALID_ARG, "bits[" + std::to_string(i) + "] = " + std::to_string(bits_host[i]) +
+                                            " outside [1, 8]");
+  }
+  cudaError_t e = cudaMemcpyAsync(c->d_bits, bits_host, table, cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "copy of schedule");
+  return TASQ_OK;
+}
+
+tasq_status tasq_linear_forward(tasq_ctx* c, const void* x, int64_t M, int64_t ldx, int32_t layer, int32_t step, void* y,
+                                int64_t ldy, void* stream) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  tasq_status st;
+  if ((st = check_layer(c, layer)) != TASQ_OK) return st;
+  if ((st = check_step(c, step)) != TASQ_OK) return st;
+  if ((st = check_tokens(c, M)) != TASQ_OK) return st;
+  const LayerInfo& L = c->layers[layer];
+  if ((st = check_rows(x, ldx, L.K, "x")) != TASQ_OK) return st;
+  if ((st = check_rows(y, ldy, L.N, "y")) != TASQ_OK) return st;
+  if ((st = check_device(c)) != TASQ_OK) return st;
+  if (M == 0) return TASQ_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  TraceRec* tr = c->trace_count < c->trace_cap ? &c->trace[c->trace_count] : nullptr;
+  if (tr) cudaEventRecord(tr->e0, s);
+  if ((st = run_prologue(c, L, x, M, ldx, c->d_xq, c->d_sx, s)) != TASQ_OK) return st;
+  if (tr) cudaEventRecord(tr->e1, s);
+  const tasq::OutKind out = c->out_dtype == TASQ_OUT_BF16 ? tasq::OutKind::BF16 : tasq::OutKind::F16;
+  if ((st = run_gemm(c, layer, step, c->d_xq, c->d_sx, M, y, ldy, out, s)) != TASQ_OK) return st;
+  if (tr) {
+    cudaEventRecord(tr->e2, s);
+    tr->ops = 2.0 * static_cast<double>(M) * L.N * L.K;
+    tr->bytes = static_cast<double>(M) * (2.0 * L.K + L.Kp + 4.0);
+    ++c->trace_count;
+  }
+  return TASQ_OK;
+}
+
+tasq_status tasq_linear_destroy(tasq_ctx* c) {
+  g_last_error.clear();
+  free_ctx(c);
+  return TASQ_OK;
+}
+
+tasq_status tasq_get_device_status(tasq_ctx* c, uint32_t* status_out, int32_t clear, void* stream) {
+  g_last_error.clear();
+  if (c == nullptr || status_out == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx or status_out is NULL");
+  tasq_status st = check_device(c);
+  if (st != TASQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, c->d_status, sizeof(v), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail_cuda(e, "read of device status");
+  if (clear) {
+    e = cudaMemsetAsync(c->d_status, 0, sizeof(uint32_t), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return fail_cuda(e, "clear of device status");
+  }
+  *status_out = v;
+  return TASQ_OK;
+}
+
+tasq_status tasq_set_wait_limit(tasq_ctx* c, uint64_t limit_ns) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  if (limit_ns < 1000ull) return fail(TASQ_ERR_INVALID_ARG, "wait limit below 1 us");
+  c->wait_limit_ns = limit_ns;
+  return TASQ_OK;
+}
+
+tasq_status tasq_layer_info(const tasq_ctx* c, int32_t layer, int32_t* N, int32_t* K, int32_t* Kp) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  tasq_status st = check_layer(c, layer);
+  if (st != TASQ_OK) return st;
+  const LayerInfo& L = c->layers[layer];
+  if (N) *N = L.N;
+  if (K) *K = L.K;
+  if (Kp) *Kp = L.Kp;
+  return TASQ_OK;
+}
+
+tasq_status tasq_debug_quantize(tasq_ctx* c, const void* x, int64_t M, int64_t ldx, int32_t layer, int8_t* xq, float* s_x,
+                                void* stream) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  tasq_status st;
+  if ((st = check_layer(c, layer)) != TASQ_OK) return st;
+  if (M < 0 || M > 0x7fffffffLL) return fail(TASQ_ERR_INVALID_ARG, "M out of range");
+  const LayerInfo& L = c->layers[layer];
+  if ((st = check_rows(x, ldx, L.K, "x")) != TASQ_OK) return st;
+  if ((st = check_rows(xq, L.Kp, L.Kp, "xq")) != TASQ_OK) return st;
+  if (s_x == nullptr || !aligned16(s_x)) return fail(TASQ_ERR_INVALID_ARG, "s_x must be a 16-byte aligned pointer");
+  if ((st = check_device(c)) != TASQ_OK) return st;
+  if (M == 0) return TASQ_OK;
+  return run_prologue(c, L, x, M, ldx, xq, s_x, static_cast<cudaStream_t>(stream));
+}
+
+tasq_status tasq_debug_gemm_s32(tasq_ctx* c, const int8_t* xq, int64_t M, int32_t layer, int32_t step, int32_t* acc,
+                                int64_t ld_acc, void* stream) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  tasq_status st;
+  if ((st = check_layer(c, layer)) != TASQ_OK) return st;
+  if ((st = check_step(c, step)) != TASQ_OK) return st;
+  if (M < 0 || M > 0x7fffffffLL) return fail(TASQ_ERR_INVALID_ARG, "M out of range");
+  const LayerInfo& L = c->layers[layer];
+  if ((st = check_rows(xq, L.Kp, L.Kp, "xq")) != TASQ_OK) return st;
+  if ((st = check_rows(acc, ld_acc, L.N, "acc")) != TASQ_OK) return st;
+  if ((st = check_device(c)) != TASQ_OK) return st;
+  if (M == 0) return TASQ_OK;
+  return run_gemm(c, layer, step, xq, nullptr, M, acc, ld_acc, tasq::OutKind::S32, static_cast<cudaStream_t>(stream));
+}
+
+tasq_status tasq_debug_gemm(tasq_ctx* c, const int8_t* xq, const float* s_x, int64_t M, int32_t layer, int32_t step,
+                            void* y, int64_t ldy, int32_t out_dtype, void* stream) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  tasq_status st;
+  if ((st = check_layer(c, layer)) != TASQ_OK) return st;
+  if ((st = check_step(c, step)) != TASQ_OK) return st;
+  if (M < 0 || M > 0x7fffffffLL) return fail(TASQ_ERR_INVALID_ARG, "M out of range");
+  if (out_dtype != TASQ_OUT_F16 && out_dtype != TASQ_OUT_BF16) return fail(TASQ_ERR_INVALID_ARG, "bad out_dtype");
+  const LayerInfo& L = c->layers[layer];
+  if ((st = check_rows(xq, L.Kp, L.Kp, "xq")) != TASQ_OK) return st;
+  if (s_x == nullptr || !aligned16(s_x)) return fail(TASQ_ERR_INVALID_ARG, "s_x must be a 16-byte aligned pointer");
+  if ((st = check_rows(y, ldy, L.N, "y")) != TASQ_OK) return st;
+  if ((st = check_device(c)) != TASQ_OK) return st;
+  if (M == 0) return TASQ_OK;
+  const tasq::OutKind out = out_dtype == TASQ_OUT_BF16 ? tasq::OutKind::BF16 : tasq::OutKind::F16;
+  return run_gemm(c, layer, step, xq, s_x, M, y, ldy, out, static_cast<cudaStream_t>(stream));
+}
+
+tasq_status tasq_debug_stuck_wait(tasq_ctx* c, void* stream) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  tasq_status st = check_device(c);
+  if (st != TASQ_OK) return st;
+  cudaError_t e = tasq::launch_stuck_wait(c->d_status, c->wait_limit_ns, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "stuck-wait launch");
+  return TASQ_OK;
+}
+
+tasq_status tasq_trace_enable(tasq_ctx* c, int32_t capacity) {
+  g_last_error.clear();
+  if (c == nullptr || capacity < 0) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL or capacity < 0");
+  tasq_status st = check_device(c);
+  if (st != TASQ_OK) return st;
+  while (static_cast<int32_t>(c->trace.size()) < capacity) {
+    TraceRec r{};
+    cudaError_t e = cudaEventCreate(&r.e0);
+    if (e == cudaSuccess) e = cudaEventCreate(&r.e1);
+    if (e == cudaSuccess) e = cudaEventCreate(&r.e2);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaEventCreate");
+    c->trace.push_back(r);
+  }
+  c->trace_cap = capacity;
+  c->trace_count = 0;
+  return TASQ_OK;
+}
+
+tasq_status tasq_trace_read(tasq_ctx* c, int32_t* prologue_launches, double* prologue_ms, int32_t* gemm_launches,
+                            double* gemm_ms, double* gemm_ops, double* prologue_bytes) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  double pm = 0, gm = 0, ops = 0, bytes = 0;
+  for (int32_t i = 0; i < c->trace_count; ++i) {
+    TraceRec& r = c->trace[i];
+    cudaError_t e = cudaEventSynchronize(r.e2);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaEventSynchronize");
+    float a = 0, b = 0;
+    e = cudaEventElapsedTime(&a, r.e0, r.e1);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&b, r.e1, r.e2);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaEventElapsedTime");
+    pm += a;
+    gm += b;
+    ops += r.ops;
+    bytes += r.bytes;
+  }
+  if (prologue_launches) *prologue_launches = c->trace_count;
+  if (gemm_launches) *gemm_launches = c->trace_count;
+  if (prologue_ms) *prologue_ms = pm;
+  if (gemm_ms) *gemm_ms = gm;
+  if (gemm_ops) *gemm_ops = ops;
+  if (prologue_bytes) *prologue_bytes = bytes;
+  c->trace_count = 0;
+  return TASQ_OK;
+}
+
+}  // extern "C"

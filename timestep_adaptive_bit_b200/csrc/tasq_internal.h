@@ -1,0 +1,52 @@
+// Launch interfaces shared by the C-ABI layer and the kernel translation units.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace tasq {
+
+// Activation prologue: block Hadamard along K, per-token absmax, RNE INT8 codes.
+struct PrologueArgs {
+  const void* x;      // FP16 [M, K], row stride ldx elements
+  int64_t ldx;
+  int32_t K;          // multiple of 8
+  int32_t Kp;         // ceil(K / n) * n
+  int64_t M;
+  int8_t* xq;         // [M, Kp]
+  float* s_x;         // [M]
+  int32_t n;          // 64 or 128
+  float sx_factor;    // fp32(1 / (127 sqrt(n)))
+};
+cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream);
+
+enum class OutKind : int { F16 = 0, BF16 = 1, S32 = 2 };
+
+// Masked INT8 GEMM: y[m, c] = sum_k xq[m, k] * mask(w[c, k]) (* s_x[m] * s_w[c]).
+struct GemmArgs {
+  int32_t M;
+  int32_t N;
+  int32_t num_kb;          // ceil(Kp / 128)
+  int32_t num_m_tiles;     // ceil(M / 256)
+  int32_t num_n_tiles;     // ceil(N / 128)
+  const uint8_t* bits_table;
+  int32_t bits_index;      // layer * num_steps + step
+  const float* s_x;
+  const float* s_w;
+  void* y;
+  int64_t ldy;
+  uint32_t* status;
+  uint64_t wait_limit_ns;
+};
+cudaError_t launch_masked_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmArgs& g,
+                               OutKind out, int num_sms, cudaStream_t stream);
+
+// Geometry of the GEMM tiles (for the host's tensor maps).
+constexpr int kGemmTileCh = 128;    // weight rows per tile
+constexpr int kGemmTileTok = 256;   // activation rows per tile
+constexpr int kGemmBlockK = 128;    // K bytes per pipeline stage
+
+cudaError_t launch_stuck_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
+
+}  // namespace tasq
