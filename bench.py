@@ -56,6 +56,9 @@ def parse_args(argv=None):
                    help="workload:layer, run a few forwards of one layer (for ncu captures) and exit")
     p.add_argument("--launches", type=int, default=3)
     p.add_argument("--bits", type=int, default=None, help="profile case: bit width (default: 5)")
+    p.add_argument("--sweep-bits", default=None,
+                   help="workload:layer, time one layer's prologue and GEMM at every bit width and exit")
+    p.add_argument("--reps", type=int, default=20)
     return p.parse_args(argv)
 
 
@@ -255,6 +258,45 @@ def profile_case(args):
     return 0 if st == 0 else 1
 
 
+def sweep_bits(args):
+    """Per-bit-width timing of one layer at full size (CUDA-event trace of each kernel)."""
+    import torch
+    import timestep_adaptive_bit_b200 as T
+    name, _, lname = args.sweep_bits.partition(":")
+    wl = workloads.WORKLOADS[name]
+    j = [n for n, _, _ in wl.block_layers].index(lname or wl.block_layers[0][0])
+    _, K, N = wl.layer_shape(j)
+    M = wl.tokens
+    dev = torch.device("cuda:0")
+    w, s_w = workloads.weights_torch(wl, j, dev)
+    s = torch.cuda.current_stream()
+    ctx = T.tasq_linear_create([(N, K, w, s_w)], 8, wl.hadamard_n, M, T.TASQ_OUT_F16, s)
+    T.tasq_set_schedule(ctx, np.array([[8, 7, 6, 5, 4, 3, 2, 1]], np.uint8), s)
+    # several input buffers so consecutive launches do not find their activations in L2
+    nbuf = max(2, int(math.ceil(3 * 126e6 / (M * K * 2))))
+    xs = [workloads.activations_torch(wl, j, dev, seed=b) for b in range(nbuf)]
+    y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    peaks, peak_kind = load_peaks()
+    out = {"sweep": f"{name}:{wl.block_layers[j][0]}", "M": M, "K": K, "N": N, "reps": args.reps, "bits": {}}
+    for step in range(8):
+        for r in range(3):
+            T.tasq_linear_forward(ctx, xs[r % nbuf], M, K, 0, step, y, N, s)
+        torch.cuda.synchronize()
+        T.tasq_trace_enable(ctx, args.reps)
+        for r in range(args.reps):
+            T.tasq_linear_forward(ctx, xs[r % nbuf], M, K, 0, step, y, N, s)
+        tr = T.tasq_trace_read(ctx)
+        g_tops = tr["gemm_ops"] / (tr["gemm_ms"] / 1e3) / 1e12
+        p_gbs = tr["prologue_bytes"] / (tr["prologue_ms"] / 1e3) / 1e9
+        out["bits"][8 - step] = {"gemm_us": 1e3 * tr["gemm_ms"] / args.reps, "gemm_tops": g_tops,
+                                 "gemm_frac_int8_burst": g_tops / (peaks["bf16_tflops"] * INT8_OVER_BF16),
+                                 "prologue_us": 1e3 * tr["prologue_ms"] / args.reps, "prologue_gbs": p_gbs,
+                                 "prologue_frac_hbm": p_gbs / peaks["hbm_gbs"]}
+    out["device_status"] = T.tasq_get_device_status(ctx)
+    print(json.dumps(out), flush=True)
+    return 0 if out["device_status"] == 0 else 1
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
@@ -273,6 +315,8 @@ def main(argv=None):
 
     if args.profile_case:
         return profile_case(args)
+    if args.sweep_bits:
+        return sweep_bits(args)
 
     dist = None
     if world > 1:

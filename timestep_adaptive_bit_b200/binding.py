@@ -220,3 +220,4 @@ def tasq_trace_read(ctx: Context) -> dict:
                                ctypes.byref(ops), ctypes.byref(pb)))
     return {"prologue_launches": pl.value, "prologue_ms": pm.value, "gemm_launches": gl.value,
             "gemm_ms": gm.value, "gemm_ops": ops.value, "prologue_bytes": pb.value}
+

@@ -10,22 +10,24 @@
 // de Hardware"). The bit width is read from the device schedule table inside the kernel, so a
 // new step needs no new weights and no different kernel.
 //
-// Design (one persistent CTA per SM, warp-specialised, 320 threads):
+// Design (one persistent CTA per SM, warp-specialised, 448 threads):
 //   tile            128 output channels x 256 tokens; the weight tile is the MMA's A operand
 //                   (M = 128), the activation-code tile its B operand (N = 256); K advances in
 //                   stages of 128 bytes = four tcgen05.mma.kind::i8 of K = 32.
-//   warp 4          TMA producer: loads the 16 KB weight tile and the 32 KB code tile of each
+//   warp 8          TMA producer: loads the 16 KB weight tile and the 32 KB code tile of each
 //                   stage into 128-byte-swizzled shared memory (4 stages in flight).
-//   warps 6-9       mask warps (only when k > 0): AND every weight byte of a landed stage with
+//   warps 10-13     mask warps (only when k > 0): AND every weight byte of a landed stage with
 //                   0xFF << k in place (layout-agnostic, 8 x 16 B per thread), fence the
 //                   generic-proxy writes to the async proxy and release the stage to the MMA.
-//   warp 5          TMEM allocation (512 columns = two 256-column INT32 accumulators) and the
+//   warp 9          TMEM allocation (512 columns = two 256-column INT32 accumulators) and the
 //                   single MMA-issuing thread; tcgen05.commit frees stages and publishes
 //                   finished accumulators.
-//   warps 0-3       epilogue: tcgen05.ld 32 lanes x 32 columns, scale, convert, store. Thread =
-//                   output channel, so a warp's store of one token row is 32 consecutive
-//                   channels. The accumulator is released as soon as it has been read, so the
-//                   MMA of the next tile overlaps the stores of this one.
+//   warps 0-7       epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (its 32 channels) and
+//                   accumulator columns 128 (w / 4) .. +127 (its 128 tokens) in chunks of 32
+//                   columns, scales, converts, writes a 32 x 32 tile into its private shared
+//                   staging buffer in output row order and stores it with one TMA bulk store.
+//                   The accumulator is released as soon as it has been read, so the MMA of the
+//                   next tile overlaps the stores of this one. Warps never wait on each other.
 // Every wait is bounded (ptx::wait_bounded); a wait that runs out records a status bit, raises
 // a CTA-wide abort flag, and every role winds down: the producer waits (bounded) for the loads
 // it issued, the MMA thread for its MMAs, then TMEM is freed and the CTA exits.
@@ -43,38 +45,51 @@ constexpr int kTileCh = kGemmTileCh;      // 128
 constexpr int kTileTok = kGemmTileTok;    // 256
 constexpr int kBlockK = kGemmBlockK;      // 128 bytes
 constexpr int kUmmaK = 32;
-constexpr int kStages = 4;
 constexpr int kABytes = kTileCh * kBlockK;
 constexpr int kBBytes = kTileTok * kBlockK;
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kAccCols = kTileTok;
 constexpr int kAccStages = 2;
 constexpr uint32_t kTmemCols = kAccCols * kAccStages;   // 512: the whole TMEM of the SM
-constexpr int kEpiWarps = 4;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kMaskWarp0 = 6;
+constexpr int kEpiWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kMaskWarp0 = 10;
 constexpr int kMaskWarps = 4;
 constexpr int kThreads = 32 * (kEpiWarps + 2 + kMaskWarps);
 constexpr int kMaskThreads = 32 * kMaskWarps;
 constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kEpiCols = kTileTok / (kEpiWarps / 4);     // 128 tokens per epilogue warp
+constexpr int kSxBytesPerWarp = kEpiCols * 4;
 
-constexpr int kBarOffset = kStages * kStageBytes;
-constexpr int kNumBars = 3 * kStages + 2 * kAccStages + 1;
-constexpr int kSmemBytes = 1024 /* alignment slack */ + kBarOffset + kNumBars * 8 + 16;
+// Shared-memory plan of one instantiation: stages of (weights, codes), the epilogue's output
+// staging (one 32 x 32 tile per warp), its s_x slices, the barriers.
+template <int OUT>
+struct Plan {
+  static constexpr int kOutBytes = OUT == static_cast<int>(OutKind::S32) ? 4 : 2;
+  static constexpr int kStages = OUT == static_cast<int>(OutKind::S32) ? 3 : 4;
+  static constexpr int kEpiStageBytes = 32 * 32 * kOutBytes;
+  static constexpr int kEpiOffset = kStages * kStageBytes;
+  static constexpr int kSxOffset = kEpiOffset + kEpiWarps * kEpiStageBytes;
+  static constexpr int kBarOffset = kSxOffset + kEpiWarps * kSxBytesPerWarp;
+  static constexpr int kNumBars = 3 * kStages + 2 * kAccStages + 1;
+  static constexpr int kSmemBytes = 1024 /* alignment slack */ + kBarOffset + kNumBars * 8 + 16;
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
 
 static_assert(kABytes % (16 * kMaskThreads) == 0, "mask pass must tile the weight stage");
 static_assert(kTileTok % 16 == 0 && kTileTok <= 256, "UMMA N");
 static_assert(kBlockK % kUmmaK == 0, "stage K");
 
+template <int STAGES>
 struct Bars {
   uint32_t base;
   __device__ uint32_t full(int s) const { return base + 8u * s; }
-  __device__ uint32_t masked(int s) const { return base + 8u * (kStages + s); }
-  __device__ uint32_t empty(int s) const { return base + 8u * (2 * kStages + s); }
-  __device__ uint32_t acc_full(int i) const { return base + 8u * (3 * kStages + i); }
-  __device__ uint32_t acc_empty(int i) const { return base + 8u * (3 * kStages + kAccStages + i); }
-  __device__ uint32_t drain() const { return base + 8u * (3 * kStages + 2 * kAccStages); }
+  __device__ uint32_t masked(int s) const { return base + 8u * (STAGES + s); }
+  __device__ uint32_t empty(int s) const { return base + 8u * (2 * STAGES + s); }
+  __device__ uint32_t acc_full(int i) const { return base + 8u * (3 * STAGES + i); }
+  __device__ uint32_t acc_empty(int i) const { return base + 8u * (3 * STAGES + kAccStages + i); }
+  __device__ uint32_t drain() const { return base + 8u * (3 * STAGES + 2 * kAccStages); }
 };
 
 __device__ __forceinline__ void raise_failure(uint32_t* status, volatile int* abort_flag, uint32_t bit) {
@@ -82,26 +97,29 @@ __device__ __forceinline__ void raise_failure(uint32_t* status, volatile int* ab
   *abort_flag = 1;
 }
 
+// y = (acc * s_x) * s_w, each product rounded once in FP32, then rounded to the output type.
 template <int OUT>
-__device__ __forceinline__ void store_out(void* y, int64_t idx, float v, uint32_t raw) {
-  if constexpr (OUT == static_cast<int>(OutKind::S32)) {
-    static_cast<int32_t*>(y)[idx] = static_cast<int32_t>(raw);
-  } else if constexpr (OUT == static_cast<int>(OutKind::F16)) {
-    static_cast<__half*>(y)[idx] = __float2half_rn(v);
+__device__ __forceinline__ uint16_t out_bits(uint32_t acc, float sx, float sw) {
+  const float v = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(acc)), sx), sw);
+  if constexpr (OUT == static_cast<int>(OutKind::F16)) {
+    return __half_as_ushort(__float2half_rn(v));
   } else {
-    static_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v);
+    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
   }
 }
 
 template <int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     masked_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
-                       const GemmArgs g) {
+                       const __grid_constant__ CUtensorMap tmap_y, const GemmArgs g) {
+  using P = Plan<OUT>;
+  constexpr int kStages = P::kStages;
+  constexpr bool kS32 = OUT == static_cast<int>(OutKind::S32);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_addr(smem);
-  const Bars bars{sbase + kBarOffset};
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarOffset + kNumBars * 8);
+  const Bars<kStages> bars{sbase + P::kBarOffset};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + P::kBarOffset + P::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -134,6 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kProducerWarp && lane == 0) {
     ptx::prefetch_tmap(&tmap_w);
     ptx::prefetch_tmap(&tmap_x);
+    ptx::prefetch_tmap(&tmap_y);
   }
   if (warp == kMmaWarp) {
     ptx::tmem_alloc(ptx::smem_addr(tmem_slot), kTmemCols);
@@ -146,6 +165,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int num_tiles = g.num_m_tiles * g.num_n_tiles;
   const uint64_t limit = g.wait_limit_ns;
+  const uint32_t a_base = sbase;
+  const uint32_t b_base = sbase + kStages * kABytes;
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
@@ -162,9 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           ptx::mbar_arrive_expect_tx(bars.full(s), kStageBytes);
-          ptx::tma_load_2d(sbase + s * kABytes, &tmap_w, bars.full(s), kb * kBlockK, nt * kTileCh);
-          ptx::tma_load_2d(sbase + kStages * kABytes + s * kBBytes, &tmap_x, bars.full(s), kb * kBlockK,
-                           mt * kTileTok);
+          ptx::tma_load_2d(a_base + s * kABytes, &tmap_w, bars.full(s), kb * kBlockK, nt * kTileCh);
+          ptx::tma_load_2d(b_base + s * kBBytes, &tmap_x, bars.full(s), kb * kBlockK, mt * kTileTok);
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
           if (++s == kStages) {
@@ -203,8 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           ptx::tc_fence_after_sync();
-          const uint64_t a_desc = ptx::smem_desc_k_sw128(sbase + s * kABytes);
-          const uint64_t b_desc = ptx::smem_desc_k_sw128(sbase + kStages * kABytes + s * kBBytes);
+          const uint64_t a_desc = ptx::smem_desc_k_sw128(a_base + s * kABytes);
+          const uint64_t b_desc = ptx::smem_desc_k_sw128(b_base + s * kBBytes);
 #pragma unroll
           for (int kk = 0; kk < kBlockK / kUmmaK; ++kk) {
             // +32 bytes along K inside the 128-byte swizzle row = +2 in the address field
@@ -263,50 +283,103 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------------------------- epilogue warps
-    const int ew = warp;  // == warp % 4: this warp may access TMEM lanes [32 ew, 32 ew + 32)
+    const int q = warp & 3;         // TMEM lanes 32 q .. 32 q + 31: channels of this warp
+    const int h = warp >> 2;        // accumulator columns 128 h .. 128 h + 127: tokens
+    uint8_t* stage = smem + P::kEpiOffset + warp * P::kEpiStageBytes;
+    const uint32_t stage_addr = ptx::smem_addr(stage);
+    float* sx_slice = reinterpret_cast<float*>(smem + P::kSxOffset + warp * kSxBytesPerWarp);
     uint32_t as = 0, aph = 0;
+    bool store_pending = false;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mt = tile % g.num_m_tiles;
       const int nt = tile / g.num_m_tiles;
+      const int tok0 = mt * kTileTok + h * kEpiCols;
       const bool got = ptx::wait_bounded(bars.acc_full(as), aph, limit, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
         if (lane == 0) raise_failure(g.status, abort_flag, TASQ_DEVICE_TIMEOUT_EPILOGUE);
         break;
       }
       ptx::tc_fence_after_sync();
-      const int ch = nt * kTileCh + ew * 32 + lane;
-      const bool ch_ok = ch < g.N;
+      const int ch = nt * kTileCh + q * 32 + lane;
       float sw = 0.0f;
-      if constexpr (OUT != static_cast<int>(OutKind::S32)) {
-        if (ch_ok) sw = g.s_w[ch];
+      if constexpr (!kS32) {
+        if (ch < g.N) sw = g.s_w[ch];
+        // this warp's 128 token scales, read once per tile into its private slice
+        float4 v4;
+        const int m = tok0 + 4 * lane;
+        v4.x = m < g.M ? g.s_x[m] : 0.0f;
+        v4.y = m + 1 < g.M ? g.s_x[m + 1] : 0.0f;
+        v4.z = m + 2 < g.M ? g.s_x[m + 2] : 0.0f;
+        v4.w = m + 3 < g.M ? g.s_x[m + 3] : 0.0f;
+        reinterpret_cast<float4*>(sx_slice)[lane] = v4;
+        __syncwarp();
       }
-      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + as * kAccCols;
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + as * kAccCols + h * kEpiCols;
 #pragma unroll 1
-      for (int chunk = 0; chunk < kTileTok / 32; ++chunk) {
+      for (int j = 0; j < kEpiCols / 32; ++j) {
         uint32_t r[32];
-        ptx::tmem_ld_32x32b_x32(tacc + chunk * 32, r);
-        ptx::tmem_ld_wait();
-        if (chunk == kTileTok / 32 - 1) {
+        ptx::tmem_ld_32x32b_x32(tacc + j * 32, r);
+        ptx::tmem_ld_wait(r);
+        if (j == kEpiCols / 32 - 1) {
           // the accumulator has been read: hand it back to the MMA before storing
           ptx::tc_fence_before_sync();
           ptx::mbar_arrive(bars.acc_empty(as));
         }
-        const int t0 = mt * kTileTok + chunk * 32;
-        if (t0 >= g.M) continue;
-        float sx_lane = 0.0f;
-        if constexpr (OUT != static_cast<int>(OutKind::S32)) {
-          if (t0 + lane < g.M) sx_lane = g.s_x[t0 + lane];
-        }
+        const int t0 = tok0 + j * 32;
+        const int c0 = nt * kTileCh + q * 32;
+        // boxes wholly past the last token or channel have nothing to store (warp-uniform)
+        if (t0 >= g.M || c0 >= g.N) continue;
+        const float4* sx4 = reinterpret_cast<const float4*>(sx_slice + j * 32);
+        if (c0 + 32 > g.N && (g.N * P::kOutBytes) % 16 != 0) {
+          // a TMA store writes whole 16-byte granules, so a box whose right edge is not 16-byte
+          // aligned would write past column N: store this one with plain predicated stores
+          const int chl = c0 + lane;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float sxj = __shfl_sync(0xffffffffu, sx_lane, j);
-          const float v = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(r[j])), sxj), sw);
-          if (ch_ok && t0 + j < g.M) store_out<OUT>(g.y, static_cast<int64_t>(t0 + j) * g.ldy + ch, v, r[j]);
+          for (int t = 0; t < 32; ++t) {
+            const float sxv = kS32 ? 0.0f : sx_slice[j * 32 + t];
+            if (chl < g.N && t0 + t < g.M) {
+              const int64_t idx = static_cast<int64_t>(t0 + t) * g.ldy + chl;
+              if constexpr (kS32) {
+                static_cast<int32_t*>(g.y)[idx] = static_cast<int32_t>(r[t]);
+              } else {
+                const uint16_t b = out_bits<OUT>(r[t], sxv, sw);
+                static_cast<uint16_t*>(g.y)[idx] = b;
+              }
+            }
+          }
+          continue;
         }
+        if (store_pending) {
+          // the previous bulk store of this warp must have finished reading the staging tile
+          if (lane == 0) ptx::bulk_wait_read0();
+          __syncwarp();
+        }
+        if constexpr (kS32) {
+          uint32_t* st = reinterpret_cast<uint32_t*>(stage);
+#pragma unroll
+          for (int t = 0; t < 32; ++t) st[t * 32 + lane] = r[t];
+        } else {
+          uint16_t* st = reinterpret_cast<uint16_t*>(stage);
+#pragma unroll
+          for (int t4 = 0; t4 < 8; ++t4) {
+            const float4 sx = sx4[t4];
+            const float sxv[4] = {sx.x, sx.y, sx.z, sx.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) st[(4 * t4 + i) * 32 + lane] = out_bits<OUT>(r[4 * t4 + i], sxv[i], sw);
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::tma_store_2d(&tmap_y, stage_addr, c0, t0);
+          ptx::bulk_commit();
+        }
+        store_pending = true;
       }
       as ^= 1u;
       if (as == 0) aph ^= 1u;
     }
+    if (lane == 0) ptx::bulk_wait0();
   }
 
   __syncwarp();
@@ -319,21 +392,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int OUT>
-cudaError_t launch_out(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& g, int num_sms,
-                       cudaStream_t stream) {
+cudaError_t launch_out(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ty, const GemmArgs& g,
+                       int num_sms, cudaStream_t stream) {
   static bool configured[64] = {false};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    e = cudaFuncSetAttribute(masked_gemm_kernel<OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    e = cudaFuncSetAttribute(masked_gemm_kernel<OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Plan<OUT>::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const int tiles = g.num_m_tiles * g.num_n_tiles;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  masked_gemm_kernel<OUT><<<grid, kThreads, kSmemBytes, stream>>>(tw, tx, g);
+  masked_gemm_kernel<OUT><<<grid, kThreads, Plan<OUT>::kSmemBytes, stream>>>(tw, tx, ty, g);
   return cudaGetLastError();
 }
 
@@ -352,13 +426,16 @@ __global__ void stuck_wait_kernel(uint32_t* status, uint64_t limit_ns) {
 
 }  // namespace
 
-cudaError_t launch_masked_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmArgs& g,
-                               OutKind out, int num_sms, cudaStream_t stream) {
+cudaError_t launch_masked_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const CUtensorMap& tmap_y,
+                               const GemmArgs& g, OutKind out, int num_sms, cudaStream_t stream) {
   if (g.M <= 0 || g.N <= 0) return cudaSuccess;
   switch (out) {
-    case OutKind::F16: return launch_out<static_cast<int>(OutKind::F16)>(tmap_w, tmap_x, g, num_sms, stream);
-    case OutKind::BF16: return launch_out<static_cast<int>(OutKind::BF16)>(tmap_w, tmap_x, g, num_sms, stream);
-    case OutKind::S32: return launch_out<static_cast<int>(OutKind::S32)>(tmap_w, tmap_x, g, num_sms, stream);
+    case OutKind::F16:
+      return launch_out<static_cast<int>(OutKind::F16)>(tmap_w, tmap_x, tmap_y, g, num_sms, stream);
+    case OutKind::BF16:
+      return launch_out<static_cast<int>(OutKind::BF16)>(tmap_w, tmap_x, tmap_y, g, num_sms, stream);
+    case OutKind::S32:
+      return launch_out<static_cast<int>(OutKind::S32)>(tmap_w, tmap_x, tmap_y, g, num_sms, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -7,12 +7,19 @@
 //   s_x = a / (127 sqrt(n))              the 2^(-k/2) normalisation folded into the scale
 //                                        (HQ-DM section 2.1, "Eficiencia de Hardware")
 //
-// One CTA of 128 threads owns one token row. Thread t holds chunks c = j * 128 + t of 8
-// consecutive channels (one 16-byte load each), so every warp load is 512 contiguous bytes.
-// A Hadamard block of n channels is n / 8 consecutive chunks, i.e. n / 8 consecutive lanes of
-// one warp: butterfly strides 1, 2, 4 run inside a thread's registers, strides 8 ... n/2 run
-// across lanes with xor shuffles. The row never leaves registers between load and store.
-// All arithmetic is FP32 round-to-nearest (no contraction: adds, subtracts and one multiply).
+// Work split: a CTA owns R consecutive token rows and R * C threads, C = Kp / 64. Thread i owns
+// the 64 consecutive channels [64 (i % C), 64 (i % C) + 64) of row i / C: 128 contiguous bytes
+// in, 64 contiguous bytes out, all 64 values in registers. R is chosen on the host so that R * C
+// fills whole warps, which keeps every lane busy for any K (the kernel is issue-bound otherwise).
+//
+// The 64 values sit in 32 register pairs, pair p = (z_p, z_(p+32)), so the butterfly stages with
+// stride 1, 2, 4, 8, 16 are packed FP32x2 add / fma (two independent IEEE round-to-nearest
+// operations each), the stride-32 stage runs inside each pair, and for n = 128 the stride-64
+// stage pairs the chunks of lanes 2j and 2j + 1 through one xor shuffle. The stages run in
+// increasing stride, each butterfly (a, b) -> (a + b, a - b) rounded once in FP32, so the codes
+// are the same bits as a textbook FP32 fast Walsh-Hadamard transform produces.
+// The per-row absmax is combined through a shared-memory atomicMax on the float bits (all values
+// are non-negative). No FMA contraction happens anywhere on the path.
 #include <cuda_fp16.h>
 
 #include "tasq_internal.h"
@@ -20,144 +27,175 @@
 namespace tasq {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kMaxRowsPerCta = 64;
+constexpr int kMaxThreads = 512;
 
-__device__ __forceinline__ uint4 ld_stream_16B(const void* p) {
+__device__ __forceinline__ uint4 ld_16B(const void* p) {
   uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
   return v;
 }
 
-__device__ __forceinline__ void st_8B(void* p, uint32_t lo, uint32_t hi) {
-  asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(lo), "r"(hi) : "memory");
+__device__ __forceinline__ void st_16B(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-__device__ __forceinline__ uint32_t quant_byte(float z, float inv) {
-  int q = __float2int_rn(__fmul_rn(z, inv));
-  q = max(-127, min(127, q));
-  return static_cast<uint32_t>(q) & 0xFFu;
+// (a + b) and (a - b), lane-wise on FP32 pairs; each result rounded once to nearest even.
+__device__ __forceinline__ void butterfly2(float2& a, float2& b) {
+  const uint64_t ua = *reinterpret_cast<const uint64_t*>(&a);
+  const uint64_t ub = *reinterpret_cast<const uint64_t*>(&b);
+  const float2 minus_one = make_float2(-1.0f, -1.0f);
+  const uint64_t um = *reinterpret_cast<const uint64_t*>(&minus_one);
+  uint64_t s, d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(s) : "l"(ua), "l"(ub));
+  // b * (-1) + a is exact in the product, so the single rounding is that of a - b
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(ub), "l"(um), "l"(ua));
+  a = *reinterpret_cast<const float2*>(&s);
+  b = *reinterpret_cast<const float2*>(&d);
 }
 
-template <int CHUNKS, int LANES_PER_BLOCK>
-__global__ void __launch_bounds__(kThreads) prologue_kernel(const PrologueArgs a) {
+__device__ __forceinline__ float2 mul2(float2 a, float s) {
+  const float2 ss = make_float2(s, s);
+  const uint64_t ua = *reinterpret_cast<const uint64_t*>(&a);
+  const uint64_t us = *reinterpret_cast<const uint64_t*>(&ss);
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(ua), "l"(us));
+  return *reinterpret_cast<const float2*>(&r);
+}
+
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+  const uint32_t lo = __byte_perm(static_cast<uint32_t>(a), static_cast<uint32_t>(b), 0x0040);
+  const uint32_t hi = __byte_perm(static_cast<uint32_t>(c), static_cast<uint32_t>(d), 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
+__device__ __forceinline__ int code(float t) {
+  int q = __float2int_rn(t);
+  return max(-127, min(127, q));
+}
+
+template <int LANES_PER_BLOCK>
+__global__ void __launch_bounds__(kMaxThreads) prologue_kernel(const PrologueArgs a, const int rows_per_cta) {
+  const int C = a.Kp >> 6;                       // 64-channel chunks per row
   const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
-  const int64_t row = blockIdx.x;
-  const int real_chunks = a.K >> 3;
-  const int all_chunks = a.Kp >> 3;
-  const __half* xr = static_cast<const __half*>(a.x) + row * a.ldx;
+  const int r_local = tid / C;
+  const int chunk = tid - r_local * C;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + r_local;
+  const bool active = r_local < rows_per_cta && row < a.M;
 
-  float v[CHUNKS][8];
-#pragma unroll
-  for (int j = 0; j < CHUNKS; ++j) {
-    const int c = j * kThreads + tid;
-    if (c < real_chunks) {
-      const uint4 u = ld_stream_16B(xr + static_cast<int64_t>(c) * 8);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        __half2 h2;
-        *reinterpret_cast<uint32_t*>(&h2) = w[i];
-        const float2 f = __half22float2(h2);
-        v[j][2 * i] = f.x;
-        v[j][2 * i + 1] = f.y;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[j][i] = 0.0f;
-    }
-  }
-
-  // butterfly stages with element stride 1, 2, 4: inside the thread
-#pragma unroll
-  for (int j = 0; j < CHUNKS; ++j) {
-#pragma unroll
-    for (int h = 1; h < 8; h <<= 1) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if ((i & h) == 0) {
-          const float lo = v[j][i];
-          const float hi = v[j][i + h];
-          v[j][i] = __fadd_rn(lo, hi);
-          v[j][i + h] = __fsub_rn(lo, hi);
-        }
-      }
-    }
-  }
-  // stages with element stride 8 m (m = 1, 2, 4 [, 8]): partner chunk sits in lane ^ m
-#pragma unroll
-  for (int m = 1; m < LANES_PER_BLOCK; m <<= 1) {
-    const bool upper = (lane & m) != 0;
-#pragma unroll
-    for (int j = 0; j < CHUNKS; ++j) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float mine = v[j][i];
-        const float other = __shfl_xor_sync(0xffffffffu, mine, m);
-        v[j][i] = upper ? __fsub_rn(other, mine) : __fadd_rn(mine, other);
-      }
-    }
-  }
-
-  // per-token absmax over the padded row (chunks past Kp are zero and do not matter)
-  float amax = 0.0f;
-#pragma unroll
-  for (int j = 0; j < CHUNKS; ++j) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[j][i]));
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  __shared__ float red[kThreads / 32];
-  if (lane == 0) red[warp] = amax;
+  __shared__ unsigned int row_max[kMaxRowsPerCta];
+  if (tid < rows_per_cta) row_max[tid] = 0u;
   __syncthreads();
-  amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
 
-  const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-  int8_t* qr = a.xq + row * a.Kp;
+  const int c0 = chunk * 64;
+  float2 v[32];
+  {
+    uint4 u[8];
+    const __half* src = static_cast<const __half*>(a.x) + row * a.ldx + c0;
 #pragma unroll
-  for (int j = 0; j < CHUNKS; ++j) {
-    const int c = j * kThreads + tid;
-    if (c < all_chunks) {
-      uint32_t lo = 0, hi = 0;
+    for (int j = 0; j < 8; ++j) {
+      u[j] = (active && c0 + 8 * j < a.K) ? ld_16B(src + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
+    }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) lo |= quant_byte(v[j][i], inv) << (8 * i);
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t lo[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+      const uint32_t hi[4] = {u[j + 4].x, u[j + 4].y, u[j + 4].z, u[j + 4].w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) hi |= quant_byte(v[j][4 + i], inv) << (8 * i);
-      st_8B(qr + static_cast<int64_t>(c) * 8, lo, hi);
+      for (int t = 0; t < 4; ++t) {
+        __half2 hl, hh;
+        *reinterpret_cast<uint32_t*>(&hl) = lo[t];
+        *reinterpret_cast<uint32_t*>(&hh) = hi[t];
+        const float2 fl = __half22float2(hl);   // channels 8j + 2t, 8j + 2t + 1
+        const float2 fh = __half22float2(hh);   // the same + 32
+        v[8 * j + 2 * t] = make_float2(fl.x, fh.x);
+        v[8 * j + 2 * t + 1] = make_float2(fl.y, fh.y);
+      }
     }
   }
-  if (tid == 0) a.s_x[row] = __fmul_rn(amax, a.sx_factor);
+
+  // strides 1, 2, 4, 8, 16: pairs p and p + h, both halves at once
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int p = 0; p < 32; ++p) {
+      if ((p & h) == 0) butterfly2(v[p], v[p + h]);
+    }
+  }
+  // stride 32: inside each pair
+#pragma unroll
+  for (int p = 0; p < 32; ++p) {
+    const float lo = v[p].x, hi = v[p].y;
+    v[p].x = __fadd_rn(lo, hi);
+    v[p].y = __fsub_rn(lo, hi);
+  }
+  // stride 64 (n = 128): the other half of the block is the chunk of lane ^ 1
+  if constexpr (LANES_PER_BLOCK == 2) {
+    const bool upper = (tid & 1) != 0;
+#pragma unroll
+    for (int p = 0; p < 32; ++p) {
+      const float ox = __shfl_xor_sync(0xffffffffu, v[p].x, 1);
+      const float oy = __shfl_xor_sync(0xffffffffu, v[p].y, 1);
+      v[p].x = upper ? __fsub_rn(ox, v[p].x) : __fadd_rn(v[p].x, ox);
+      v[p].y = upper ? __fsub_rn(oy, v[p].y) : __fadd_rn(v[p].y, oy);
+    }
+  }
+
+  float m = 0.0f;
+#pragma unroll
+  for (int p = 0; p < 32; ++p) m = fmaxf(m, fmaxf(fabsf(v[p].x), fabsf(v[p].y)));
+  if (active) atomicMax(&row_max[r_local], __float_as_uint(m));
+  __syncthreads();
+  if (!active) return;
+  const float amax = __uint_as_float(row_max[r_local]);
+  const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+
+#pragma unroll
+  for (int p = 0; p < 32; ++p) v[p] = mul2(v[p], inv);
+  uint32_t w[16];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {   // bytes 4j .. 4j + 3 are channels 4j .. 4j + 3 (low half)
+    w[j] = pack4(code(v[4 * j].x), code(v[4 * j + 1].x), code(v[4 * j + 2].x), code(v[4 * j + 3].x));
+    w[8 + j] = pack4(code(v[4 * j].y), code(v[4 * j + 1].y), code(v[4 * j + 2].y), code(v[4 * j + 3].y));
+  }
+  int8_t* dst = a.xq + row * a.Kp + c0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) st_16B(dst + 16 * j, w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  if (chunk == 0) a.s_x[row] = __fmul_rn(amax, a.sx_factor);
 }
 
-template <int LPB>
-cudaError_t launch_for_chunks(int chunks, const PrologueArgs& a, cudaStream_t s) {
-  const dim3 grid(static_cast<unsigned>(a.M)), block(kThreads);
-  switch (chunks) {
-    case 1: prologue_kernel<1, LPB><<<grid, block, 0, s>>>(a); break;
-    case 2: prologue_kernel<2, LPB><<<grid, block, 0, s>>>(a); break;
-    case 3: prologue_kernel<3, LPB><<<grid, block, 0, s>>>(a); break;
-    case 4: prologue_kernel<4, LPB><<<grid, block, 0, s>>>(a); break;
-    case 5: case 6: prologue_kernel<6, LPB><<<grid, block, 0, s>>>(a); break;
-    case 7: case 8: prologue_kernel<8, LPB><<<grid, block, 0, s>>>(a); break;
-    case 9: case 10: case 11: case 12: prologue_kernel<12, LPB><<<grid, block, 0, s>>>(a); break;
-    case 13: case 14: case 15: case 16: prologue_kernel<16, LPB><<<grid, block, 0, s>>>(a); break;
-    default: return cudaErrorInvalidValue;
+// rows per CTA: fill whole warps (R * C a multiple of 32) with 128..512 threads where possible
+int pick_rows(int C) {
+  int best_r = 1;
+  double best_score = -1.0;
+  for (int r = 1; r <= kMaxRowsPerCta && r * C <= kMaxThreads; ++r) {
+    const int t = r * C;
+    const double util = static_cast<double>(t) / (((t + 31) / 32) * 32);
+    double score = util;
+    if (t < 128) score -= 0.05 * (128 - t) / 128.0;
+    if (score > best_score + 1e-9) {
+      best_score = score;
+      best_r = r;
+    }
   }
-  return cudaGetLastError();
+  return best_r;
 }
 
 }  // namespace
 
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
   if (a.M <= 0) return cudaSuccess;
-  const int chunks = (a.Kp / 8 + kThreads - 1) / kThreads;
-  if (a.n == 64) return launch_for_chunks<8>(chunks, a, stream);
-  if (a.n == 128) return launch_for_chunks<16>(chunks, a, stream);
-  return cudaErrorInvalidValue;
+  if (a.Kp % 64 != 0 || (a.n != 64 && a.n != 128)) return cudaErrorInvalidValue;
+  const int C = a.Kp / 64;
+  if (C > kMaxThreads) return cudaErrorInvalidValue;
+  const int R = pick_rows(C);
+  const int threads = ((R * C + 31) / 32) * 32;
+  const int64_t grid = (a.M + R - 1) / R;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+  if (a.n == 64)
+    prologue_kernel<1><<<static_cast<unsigned>(grid), threads, 0, stream>>>(a, R);
+  else
+    prologue_kernel<2><<<static_cast<unsigned>(grid), threads, 0, stream>>>(a, R);
+  return cudaGetLastError();
 }
 
 }  // namespace tasq

@@ -14,9 +14,12 @@
 #include "../../include/tasq.h"
 #include "tasq_internal.h"
 
-namespace {
+namespace tasq {
 
 thread_local std::string g_last_error;
+
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+
 
 tasq_status fail(tasq_status st, const std::string& msg) {
   g_last_error = msg;
@@ -61,6 +64,35 @@ tasq_status make_tmap_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64
   if (r != CUDA_SUCCESS) return fail(TASQ_ERR_CUDA, "cuTensorMapEncodeTiled failed with CUresult " + std::to_string(r));
   return TASQ_OK;
 }
+
+// 2-D output tensor [rows, cols] (element type `dt`, row stride `ld` elements) written in
+// boxes of 32 x 32 by TMA stores; elements outside [rows, cols] are never written.
+tasq_status make_tmap_out(CUtensorMap* m, void* base, CUtensorMapDataType dt, uint32_t elem_bytes, uint64_t cols,
+                          uint64_t rows, uint64_t ld) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(TASQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {ld * elem_bytes};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(tasq::kGemmStoreBox), static_cast<cuuint32_t>(tasq::kGemmStoreBox)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(TASQ_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed with CUresult " + std::to_string(r));
+  return TASQ_OK;
+}
+
+}  // namespace tasq
+
+namespace {
+
+using tasq::fail;
+using tasq::fail_cuda;
+using tasq::aligned16;
+using tasq::round_up;
+using tasq::make_tmap_u8;
+using tasq::make_tmap_out;
+using tasq::g_last_error;
 
 struct LayerInfo {
   int32_t N, K, Kp;
@@ -181,6 +213,13 @@ tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq,
   tasq_status st = make_tmap_u8(&tx, xq, static_cast<uint64_t>(L.Kp), static_cast<uint64_t>(M), tasq::kGemmBlockK,
                                 tasq::kGemmTileTok);
   if (st != TASQ_OK) return st;
+  CUtensorMap ty;
+  const CUtensorMapDataType dt = out == tasq::OutKind::S32    ? CU_TENSOR_MAP_DATA_TYPE_INT32
+                                 : out == tasq::OutKind::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const uint32_t eb = out == tasq::OutKind::S32 ? 4u : 2u;
+  st = make_tmap_out(&ty, y, dt, eb, static_cast<uint64_t>(L.N), static_cast<uint64_t>(M), static_cast<uint64_t>(ldy));
+  if (st != TASQ_OK) return st;
   tasq::GemmArgs g{};
   g.M = static_cast<int32_t>(M);
   g.N = L.N;
@@ -195,7 +234,7 @@ tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq,
   g.ldy = ldy;
   g.status = c->d_status;
   g.wait_limit_ns = c->wait_limit_ns;
-  cudaError_t e = tasq::launch_masked_gemm(c->tmap_w[layer], tx, g, out, c->num_sms, s);
+  cudaError_t e = tasq::launch_masked_gemm(c->tmap_w[layer], tx, ty, g, out, c->num_sms, s);
   if (e != cudaSuccess) return fail_cuda(e, "masked GEMM launch");
   return TASQ_OK;
 }

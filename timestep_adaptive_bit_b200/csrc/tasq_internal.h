@@ -2,8 +2,12 @@
 #pragma once
 
 #include <cstdint>
+#include <string>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
+
+#include "../../include/tasq.h"
 
 namespace tasq {
 
@@ -39,14 +43,29 @@ struct GemmArgs {
   uint32_t* status;
   uint64_t wait_limit_ns;
 };
-cudaError_t launch_masked_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmArgs& g,
-                               OutKind out, int num_sms, cudaStream_t stream);
+cudaError_t launch_masked_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const CUtensorMap& tmap_y,
+                               const GemmArgs& g, OutKind out, int num_sms, cudaStream_t stream);
 
 // Geometry of the GEMM tiles (for the host's tensor maps).
 constexpr int kGemmTileCh = 128;    // weight rows per tile
 constexpr int kGemmTileTok = 256;   // activation rows per tile
 constexpr int kGemmBlockK = 128;    // K bytes per pipeline stage
+constexpr int kGemmStoreBox = 32;   // outputs leave in 32 x 32 TMA store boxes
 
 cudaError_t launch_stuck_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
+
+// Host helpers shared by the entry points (defined in tasq_api.cu).
+extern thread_local std::string g_last_error;
+void set_last_error(const std::string& msg);
+tasq_status fail(tasq_status st, const std::string& msg);
+tasq_status fail_cuda(cudaError_t e, const char* what);
+bool aligned16(const void* p);
+size_t round_up(size_t v, size_t a);
+// UINT8 [rows, cols] tensor (row stride cols bytes) read in 128-byte-swizzled boxes.
+tasq_status make_tmap_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                         uint32_t box_rows);
+// Output tensor [rows, cols] (row stride ld elements) written in 32 x 32 boxes.
+tasq_status make_tmap_out(CUtensorMap* m, void* base, CUtensorMapDataType dt, uint32_t elem_bytes, uint64_t cols,
+                          uint64_t rows, uint64_t ld);
 
 }  // namespace tasq
