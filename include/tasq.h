@@ -182,6 +182,37 @@ tasq_status tasq_trace_enable(tasq_ctx* ctx, int32_t capacity);
 tasq_status tasq_trace_read(tasq_ctx* ctx, int32_t* prologue_launches, double* prologue_ms,
                             int32_t* gemm_launches, double* gemm_ms, double* gemm_ops, double* prologue_bytes);
 
+/*
+ * Allocation-free variant of tasq_linear_forward, for callers that cannot call cudaMalloc:
+ * code that runs inside a custom allocator or memory-pool callback, a host that hands every byte
+ * of device memory to its own arena up front, or a capture harness that forbids allocation.
+ * The pages have no counterpart; this is a deployment entry point around the same two kernels.
+ *
+ * No context is needed: the caller passes the layer's weights directly (the mask is applied to
+ * them in flight, they are never copied or modified) and this call allocates nothing. The
+ * activation codes and scales go to one fixed device array of TASQ_NOALLOC_SCRATCH_BYTES that
+ * every GPU loading this library reserves until the process exits.
+ *   x          : device FP16 [M, K], row stride ldx (>= K, % 8 == 0), 16-byte aligned.
+ *   K          : in-features, >= 8 and % 8 == 0; Kp = ceil(K / hadamard_n) * hadamard_n.
+ *   w          : device INT8 [N, Kp] row-major, 16-byte aligned (caller-owned, read only).
+ *   s_w        : device FP32 [N].
+ *   bits       : bit width for this call, 1..8 (8 = all bit planes kept).
+ *   y          : device [M, N] in out_dtype, row stride ldy (>= N, % 8 == 0), 16-byte aligned.
+ *   device_status : optional device uint32 that receives TASQ_DEVICE_* bits (OR-ed in; the
+ *                caller clears it); NULL sends them to a word inside the fixed array.
+ * Limits: (M * 4 rounded up to 1 KiB) + 256 + M * Kp must not exceed TASQ_NOALLOC_SCRATCH_BYTES;
+ * larger sizes return TASQ_ERR_WORKSPACE before anything is enqueued.
+ * The first call on each device, made with that device current, looks the array's device
+ * address up (cudaGetSymbolAddress) and caches it; make that first call before any stream
+ * capture. Every call uses the same array and leaves its contents behind for the next one, so
+ * calls that overlap on the GPU (on different streams, or from different threads without
+ * ordering) race on it and must be serialised by the caller.
+ */
+#define TASQ_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+tasq_status tasq_linear_forward_noalloc(const void* x, int64_t M, int64_t ldx, int32_t K, const int8_t* w,
+                                        const float* s_w, int32_t N, int32_t bits, int32_t hadamard_n, void* y,
+                                        int64_t ldy, int32_t out_dtype, uint32_t* device_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

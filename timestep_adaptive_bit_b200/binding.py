@@ -35,6 +35,7 @@ TASQ_DEVICE_TIMEOUT_DRAIN = 0x10
 TASQ_DEVICE_BAD_BITS = 0x100
 
 TASQ_MAX_KP = 16384
+TASQ_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
 class TasqError(RuntimeError):
@@ -69,6 +70,7 @@ def _load():
         "tasq_debug_gemm": [P, P, P, i64, i32, i32, P, i64, i32, P],
         "tasq_debug_stuck_wait": [P, P],
         "tasq_trace_enable": [P, i32],
+        "tasq_linear_forward_noalloc": [P, i64, i64, i32, P, P, i32, i32, i32, P, i64, i32, P, P],
         "tasq_trace_read": [P, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i32),
                             ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
                             ctypes.POINTER(ctypes.c_double)],
@@ -221,3 +223,11 @@ def tasq_trace_read(ctx: Context) -> dict:
     return {"prologue_launches": pl.value, "prologue_ms": pm.value, "gemm_launches": gl.value,
             "gemm_ms": gm.value, "gemm_ops": ops.value, "prologue_bytes": pb.value}
 
+
+def tasq_linear_forward_noalloc(x, M: int, ldx: int, K: int, w, s_w, N: int, bits: int, hadamard_n: int, y,
+                                ldy: int, out_dtype: int = TASQ_OUT_F16, device_status=None, stream=None) -> None:
+    """Allocation-free forward: no context, the caller's weights are used in place and the
+    activation workspace is a fixed device array inside the library (see include/tasq.h)."""
+    _check(lib.tasq_linear_forward_noalloc(_ptr(x), int(M), int(ldx), int(K), _ptr(w), _ptr(s_w), int(N), int(bits),
+                                           int(hadamard_n), _ptr(y), int(ldy), int(out_dtype), _ptr(device_status),
+                                           _stream(stream)))
