@@ -7,16 +7,17 @@
 //   s_x = a / (127 sqrt(n))              the 2^(-k/2) normalisation folded into the scale
 //                                        (HQ-DM section 2.1, "Eficiencia de Hardware")
 //
-// Work split: a CTA owns R consecutive token rows and R * C threads, C = Kp / 64. Thread i owns
-// the 64 consecutive channels [64 (i % C), 64 (i % C) + 64) of row i / C: 128 contiguous bytes
-// in, 64 contiguous bytes out, all 64 values in registers. R is chosen on the host so that R * C
-// fills whole warps, which keeps every lane busy for any K (the kernel is issue-bound otherwise).
+// Work split: a CTA owns R consecutive token rows and R * L threads, L = Kp / 32. Thread i owns
+// the 32 consecutive channels [32 (i % L), 32 (i % L) + 32) of row i / L: 64 contiguous bytes in
+// (two full 32-byte sectors), 32 contiguous bytes out (one sector), all values in registers. A
+// Hadamard block of n channels is n / 32 neighbouring lanes. R is chosen on the host so that R * L
+// fills whole warps, which keeps every lane busy for any K.
 //
-// The 64 values sit in 32 register pairs, pair p = (z_p, z_(p+32)), so the butterfly stages with
-// stride 1, 2, 4, 8, 16 are packed FP32x2 add / fma (two independent IEEE round-to-nearest
-// operations each), the stride-32 stage runs inside each pair, and for n = 128 the stride-64
-// stage pairs the chunks of lanes 2j and 2j + 1 through one xor shuffle. The stages run in
-// increasing stride, each butterfly (a, b) -> (a + b, a - b) rounded once in FP32, so the codes
+// The 32 values sit in 16 register pairs, pair p = (z_p, z_(p+16)), so the butterfly stages with
+// stride 1, 2, 4, 8 are packed FP32x2 add / fma (two independent IEEE round-to-nearest operations
+// each), the stride-16 stage runs inside each pair, and the stride-32 (and, for n = 128,
+// stride-64) stage pairs lane i with lane i ^ 1 (and i ^ 2) through xor shuffles. The stages run
+// in increasing stride, each butterfly (a, b) -> (a + b, a - b) rounded once in FP32, so the codes
 // are the same bits as a textbook FP32 fast Walsh-Hadamard transform produces.
 // The per-row absmax is combined through a shared-memory atomicMax on the float bits (all values
 // are non-negative). No FMA contraction happens anywhere on the path.
@@ -36,8 +37,27 @@ __device__ __forceinline__ uint4 ld_16B(const void* p) {
   return v;
 }
 
+// 32-byte load (one full sector); the address must be 32-byte aligned.
+__device__ __forceinline__ void ld_32B(const void* p, uint32_t (&u)[8]) {
+  float f[8];
+  asm volatile("ld.global.L1::no_allocate.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3]), "=f"(f[4]), "=f"(f[5]), "=f"(f[6]), "=f"(f[7])
+               : "l"(p));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) u[i] = __float_as_uint(f[i]);
+}
+
 __device__ __forceinline__ void st_16B(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// 32-byte store (one full sector); the address must be 32-byte aligned.
+__device__ __forceinline__ void st_32B(void* p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.L1::no_allocate.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
+               "f"(__uint_as_float(w[0])), "f"(__uint_as_float(w[1])), "f"(__uint_as_float(w[2])),
+               "f"(__uint_as_float(w[3])), "f"(__uint_as_float(w[4])), "f"(__uint_as_float(w[5])),
+               "f"(__uint_as_float(w[6])), "f"(__uint_as_float(w[7]))
+               : "memory");
 }
 
 // (a + b) and (a - b), lane-wise on FP32 pairs; each result rounded once to nearest even.
@@ -74,12 +94,13 @@ __device__ __forceinline__ int code(float t) {
   return max(-127, min(127, q));
 }
 
-template <int LANES_PER_BLOCK>
+// LANES = n / 32 lanes per Hadamard block; VEC32: row starts of x and xq are 32-byte aligned.
+template <int LANES, bool VEC32>
 __global__ void __launch_bounds__(kMaxThreads) prologue_kernel(const PrologueArgs a, const int rows_per_cta) {
-  const int C = a.Kp >> 6;                       // 64-channel chunks per row
+  const int L = a.Kp >> 5;                       // 32-channel segments per row
   const int tid = threadIdx.x;
-  const int r_local = tid / C;
-  const int chunk = tid - r_local * C;
+  const int r_local = tid / L;
+  const int seg = tid - r_local * L;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + r_local;
   const bool active = r_local < rows_per_cta && row < a.M;
 
@@ -87,80 +108,100 @@ __global__ void __launch_bounds__(kMaxThreads) prologue_kernel(const PrologueArg
   if (tid < rows_per_cta) row_max[tid] = 0u;
   __syncthreads();
 
-  const int c0 = chunk * 64;
-  float2 v[32];
+  const int c0 = seg * 32;
+  float2 v[16];
   {
-    uint4 u[8];
+    uint32_t u[16];   // u[i] holds channels c0 + 2i, c0 + 2i + 1
     const __half* src = static_cast<const __half*>(a.x) + row * a.ldx + c0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      u[j] = (active && c0 + 8 * j < a.K) ? ld_16B(src + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
+    for (int g = 0; g < 2; ++g) {
+      uint32_t* ug = u + 8 * g;
+      const int e0 = c0 + 16 * g;
+      if (active && e0 + 16 <= a.K) {
+        if constexpr (VEC32) {
+          uint32_t t[8];
+          ld_32B(src + 16 * g, t);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) ug[i] = t[i];
+        } else {
+          const uint4 p0 = ld_16B(src + 16 * g), p1 = ld_16B(src + 16 * g + 8);
+          ug[0] = p0.x; ug[1] = p0.y; ug[2] = p0.z; ug[3] = p0.w;
+          ug[4] = p1.x; ug[5] = p1.y; ug[6] = p1.z; ug[7] = p1.w;
+        }
+      } else if (active && e0 + 8 <= a.K) {
+        const uint4 p0 = ld_16B(src + 16 * g);
+        ug[0] = p0.x; ug[1] = p0.y; ug[2] = p0.z; ug[3] = p0.w;
+        ug[4] = 0u; ug[5] = 0u; ug[6] = 0u; ug[7] = 0u;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ug[i] = 0u;
+      }
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t lo[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
-      const uint32_t hi[4] = {u[j + 4].x, u[j + 4].y, u[j + 4].z, u[j + 4].w};
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        __half2 hl, hh;
-        *reinterpret_cast<uint32_t*>(&hl) = lo[t];
-        *reinterpret_cast<uint32_t*>(&hh) = hi[t];
-        const float2 fl = __half22float2(hl);   // channels 8j + 2t, 8j + 2t + 1
-        const float2 fh = __half22float2(hh);   // the same + 32
-        v[8 * j + 2 * t] = make_float2(fl.x, fh.x);
-        v[8 * j + 2 * t + 1] = make_float2(fl.y, fh.y);
-      }
+    for (int i = 0; i < 8; ++i) {
+      __half2 hl, hh;
+      *reinterpret_cast<uint32_t*>(&hl) = u[i];       // channels 2i, 2i + 1
+      *reinterpret_cast<uint32_t*>(&hh) = u[i + 8];   // channels 16 + 2i, 17 + 2i
+      const float2 fl = __half22float2(hl);
+      const float2 fh = __half22float2(hh);
+      v[2 * i] = make_float2(fl.x, fh.x);
+      v[2 * i + 1] = make_float2(fl.y, fh.y);
     }
   }
 
-  // strides 1, 2, 4, 8, 16: pairs p and p + h, both halves at once
+  // strides 1, 2, 4, 8: pairs p and p + h, both halves at once
 #pragma unroll
-  for (int h = 1; h < 32; h <<= 1) {
+  for (int h = 1; h < 16; h <<= 1) {
 #pragma unroll
-    for (int p = 0; p < 32; ++p) {
+    for (int p = 0; p < 16; ++p) {
       if ((p & h) == 0) butterfly2(v[p], v[p + h]);
     }
   }
-  // stride 32: inside each pair
+  // stride 16: inside each pair
 #pragma unroll
-  for (int p = 0; p < 32; ++p) {
+  for (int p = 0; p < 16; ++p) {
     const float lo = v[p].x, hi = v[p].y;
     v[p].x = __fadd_rn(lo, hi);
     v[p].y = __fsub_rn(lo, hi);
   }
-  // stride 64 (n = 128): the other half of the block is the chunk of lane ^ 1
-  if constexpr (LANES_PER_BLOCK == 2) {
-    const bool upper = (tid & 1) != 0;
+  // strides 32 (and 64): the partner segment of the block sits in lane ^ m
 #pragma unroll
-    for (int p = 0; p < 32; ++p) {
-      const float ox = __shfl_xor_sync(0xffffffffu, v[p].x, 1);
-      const float oy = __shfl_xor_sync(0xffffffffu, v[p].y, 1);
+  for (int m = 1; m < LANES; m <<= 1) {
+    const bool upper = (seg & m) != 0;
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      const float ox = __shfl_xor_sync(0xffffffffu, v[p].x, m);
+      const float oy = __shfl_xor_sync(0xffffffffu, v[p].y, m);
       v[p].x = upper ? __fsub_rn(ox, v[p].x) : __fadd_rn(v[p].x, ox);
       v[p].y = upper ? __fsub_rn(oy, v[p].y) : __fadd_rn(v[p].y, oy);
     }
   }
 
-  float m = 0.0f;
+  float mx = 0.0f;
 #pragma unroll
-  for (int p = 0; p < 32; ++p) m = fmaxf(m, fmaxf(fabsf(v[p].x), fabsf(v[p].y)));
-  if (active) atomicMax(&row_max[r_local], __float_as_uint(m));
+  for (int p = 0; p < 16; ++p) mx = fmaxf(mx, fmaxf(fabsf(v[p].x), fabsf(v[p].y)));
+  if (active) atomicMax(&row_max[r_local], __float_as_uint(mx));
   __syncthreads();
   if (!active) return;
   const float amax = __uint_as_float(row_max[r_local]);
   const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
 
 #pragma unroll
-  for (int p = 0; p < 32; ++p) v[p] = mul2(v[p], inv);
-  uint32_t w[16];
+  for (int p = 0; p < 16; ++p) v[p] = mul2(v[p], inv);
+  uint32_t w[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {   // bytes 4j .. 4j + 3 are channels 4j .. 4j + 3 (low half)
+  for (int j = 0; j < 4; ++j) {   // bytes 4j .. 4j + 3 are channels 4j .. 4j + 3
     w[j] = pack4(code(v[4 * j].x), code(v[4 * j + 1].x), code(v[4 * j + 2].x), code(v[4 * j + 3].x));
-    w[8 + j] = pack4(code(v[4 * j].y), code(v[4 * j + 1].y), code(v[4 * j + 2].y), code(v[4 * j + 3].y));
+    w[4 + j] = pack4(code(v[4 * j].y), code(v[4 * j + 1].y), code(v[4 * j + 2].y), code(v[4 * j + 3].y));
   }
   int8_t* dst = a.xq + row * a.Kp + c0;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) st_16B(dst + 16 * j, w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-  if (chunk == 0) a.s_x[row] = __fmul_rn(amax, a.sx_factor);
+  if constexpr (VEC32) {
+    st_32B(dst, w);
+  } else {
+    st_16B(dst, w[0], w[1], w[2], w[3]);
+    st_16B(dst + 16, w[4], w[5], w[6], w[7]);
+  }
+  if (seg == 0) a.s_x[row] = __fmul_rn(amax, a.sx_factor);
 }
 
 // rows per CTA: fill whole warps (R * C a multiple of 32) with 128..512 threads where possible
@@ -184,17 +225,23 @@ int pick_rows(int C) {
 
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
   if (a.M <= 0) return cudaSuccess;
-  if (a.Kp % 64 != 0 || (a.n != 64 && a.n != 128)) return cudaErrorInvalidValue;
-  const int C = a.Kp / 64;
-  if (C > kMaxThreads) return cudaErrorInvalidValue;
-  const int R = pick_rows(C);
-  const int threads = ((R * C + 31) / 32) * 32;
+  if (a.Kp % a.n != 0 || (a.n != 64 && a.n != 128)) return cudaErrorInvalidValue;
+  const int L = a.Kp / 32;
+  if (L > kMaxThreads) return cudaErrorInvalidValue;
+  const int R = pick_rows(L);
+  const int threads = ((R * L + 31) / 32) * 32;
   const int64_t grid = (a.M + R - 1) / R;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
-  if (a.n == 64)
-    prologue_kernel<1><<<static_cast<unsigned>(grid), threads, 0, stream>>>(a, R);
-  else
-    prologue_kernel<2><<<static_cast<unsigned>(grid), threads, 0, stream>>>(a, R);
+  const bool vec32 = (reinterpret_cast<uintptr_t>(a.x) % 32 == 0) && (a.ldx % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(a.xq) % 32 == 0);
+  const unsigned gx = static_cast<unsigned>(grid);
+  if (a.n == 64) {
+    if (vec32) prologue_kernel<2, true><<<gx, threads, 0, stream>>>(a, R);
+    else prologue_kernel<2, false><<<gx, threads, 0, stream>>>(a, R);
+  } else {
+    if (vec32) prologue_kernel<4, true><<<gx, threads, 0, stream>>>(a, R);
+    else prologue_kernel<4, false><<<gx, threads, 0, stream>>>(a, R);
+  }
   return cudaGetLastError();
 }
 
