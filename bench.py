@@ -59,6 +59,8 @@ def parse_args(argv=None):
     p.add_argument("--sweep-bits", default=None,
                    help="workload:layer, time one layer's prologue and GEMM at every bit width and exit")
     p.add_argument("--reps", type=int, default=20)
+    p.add_argument("--gemm-mode", type=int, default=0, choices=[0, 1, 2],
+                   help="GEMM kernel: 0 automatic, 1 one CTA per tile, 2 CTA pairs")
     return p.parse_args(argv)
 
 
@@ -245,6 +247,7 @@ def profile_case(args):
     w, s_w = workloads.weights_torch(wl, j, dev)
     s = torch.cuda.current_stream()
     ctx = T.tasq_linear_create([(N, K, w, s_w)], 1, wl.hadamard_n, wl.tokens, T.TASQ_OUT_F16, s)
+    T.tasq_debug_set_gemm_mode(ctx, args.gemm_mode)
     bits = 5 if args.bits is None else args.bits
     T.tasq_set_schedule(ctx, np.array([[bits]], np.uint8), s)
     x = workloads.activations_torch(wl, j, dev)
@@ -271,13 +274,15 @@ def sweep_bits(args):
     w, s_w = workloads.weights_torch(wl, j, dev)
     s = torch.cuda.current_stream()
     ctx = T.tasq_linear_create([(N, K, w, s_w)], 8, wl.hadamard_n, M, T.TASQ_OUT_F16, s)
+    T.tasq_debug_set_gemm_mode(ctx, args.gemm_mode)
     T.tasq_set_schedule(ctx, np.array([[8, 7, 6, 5, 4, 3, 2, 1]], np.uint8), s)
     # several input buffers so consecutive launches do not find their activations in L2
     nbuf = max(2, int(math.ceil(3 * 126e6 / (M * K * 2))))
     xs = [workloads.activations_torch(wl, j, dev, seed=b) for b in range(nbuf)]
     y = torch.empty((M, N), dtype=torch.float16, device=dev)
     peaks, peak_kind = load_peaks()
-    out = {"sweep": f"{name}:{wl.block_layers[j][0]}", "M": M, "K": K, "N": N, "reps": args.reps, "bits": {}}
+    out = {"sweep": f"{name}:{wl.block_layers[j][0]}", "M": M, "K": K, "N": N, "reps": args.reps,
+           "gemm_mode": args.gemm_mode, "bits": {}}
     for step in range(8):
         for r in range(3):
             T.tasq_linear_forward(ctx, xs[r % nbuf], M, K, 0, step, y, N, s)

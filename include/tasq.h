@@ -164,6 +164,14 @@ tasq_status tasq_debug_gemm(tasq_ctx* ctx, const int8_t* xq, const float* s_x, i
                             int32_t step, void* y, int64_t ldy, int32_t out_dtype, void* stream);
 
 /*
+ * Test hook: which GEMM kernel later forwards of this context use. 0 (default) lets the library
+ * choose per launch from the wave count of each kernel's tiles, 1 forces one CTA per 128 x 256
+ * tile (tcgen05 cta_group::1), 2 forces CTA pairs on 256 x 256 tiles (tcgen05 cta_group::2).
+ * Both compute identical results.
+ */
+tasq_status tasq_debug_set_gemm_mode(tasq_ctx* ctx, int32_t mode);
+
+/*
  * Failure-detection hook: launch one CTA that waits, with the context's wait limit, on a
  * shared-memory barrier that nothing ever arrives on. The wait must run out, set
  * TASQ_DEVICE_TIMEOUT_MMA in the status word and return. Used by tests to check that a

@@ -93,15 +93,22 @@ def test_prologue_matches_oracle(T, n, K, M):
 
 
 # ----------------------------------------------------------------------------- GEMM, exact
+# GEMM kernels: 1 = one CTA per 128 x 256 tile, 2 = CTA pairs on 256 x 256 tiles
+GEMM_MODES = [1, 2]
+
+
+@pytest.mark.parametrize("mode", GEMM_MODES)
 @pytest.mark.parametrize("M,N,K,n", [(1, 1, 64, 64), (256, 128, 128, 64), (300, 200, 1152, 64), (513, 384, 192, 64),
-                                     (100, 1152, 2240, 128), (257, 130, 4608, 64), (64, 2000, 64, 64)])
-def test_gemm_s32_bit_exact_all_bits(T, M, N, K, n):
+                                     (100, 1152, 2240, 128), (257, 130, 4608, 64), (64, 2000, 64, 64),
+                                     (700, 520, 320, 64)])
+def test_gemm_s32_bit_exact_all_bits(T, M, N, K, n, mode):
     rng = np.random.default_rng(M * 7 + N * 13 + K)
     Kp = oracle.padded_k(K, n)
     w = rng.integers(-128, 128, size=(N, Kp)).astype(np.int8)     # includes -128
     q = rng.integers(-127, 128, size=(M, Kp)).astype(np.int8)
     steps = 8
     ctx = _ctx(T, [(N, K, w, np.ones(N, np.float32))], steps, n, M)
+    T.tasq_debug_set_gemm_mode(ctx, mode)
     bits = np.array([[8, 7, 6, 5, 4, 3, 2, 1]], np.uint8)
     T.tasq_set_schedule(ctx, bits, _stream())
     qd = _dev(q)
@@ -117,7 +124,8 @@ def test_gemm_s32_bit_exact_all_bits(T, M, N, K, n):
     assert T.tasq_get_device_status(ctx) == 0
 
 
-def test_gemm_extreme_values(T):
+@pytest.mark.parametrize("mode", GEMM_MODES)
+def test_gemm_extreme_values(T, mode):
     """All-(-128) weights at k = 0 and all-(-127) codes: the largest accumulators at Kp = 12288."""
     M, N, K = 256, 128, 12288
     w = np.full((N, K), -128, np.int8)
@@ -125,6 +133,7 @@ def test_gemm_extreme_values(T):
     q = np.full((M, K), -127, np.int8)
     q[::3] = 127
     ctx = _ctx(T, [(N, K, w, np.ones(N, np.float32))], 2, 64, M)
+    T.tasq_debug_set_gemm_mode(ctx, mode)
     T.tasq_set_schedule(ctx, np.array([[8, 1]], np.uint8), _stream())
     acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
     for step, bits in ((0, 8), (1, 1)):
@@ -135,9 +144,10 @@ def test_gemm_extreme_values(T):
 
 
 # ----------------------------------------------------------------------------- dequant epilogue
+@pytest.mark.parametrize("mode", GEMM_MODES)
 @pytest.mark.parametrize("out", [0, 1])
 @pytest.mark.parametrize("M,N,K", [(300, 200, 1152), (17, 1152, 64), (512, 256, 256)])
-def test_gemm_dequant_given_codes(T, out, M, N, K):
+def test_gemm_dequant_given_codes(T, out, M, N, K, mode):
     rng = np.random.default_rng(M + N + K + out)
     w = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
     s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
@@ -145,6 +155,7 @@ def test_gemm_dequant_given_codes(T, out, M, N, K):
     s_x = rng.uniform(0.01, 3.0, size=M).astype(np.float32)
     s_x[0] = 0.0
     ctx = _ctx(T, [(N, K, w, s_w)], 2, 64, M)
+    T.tasq_debug_set_gemm_mode(ctx, mode)
     T.tasq_set_schedule(ctx, np.array([[8, 5]], np.uint8), _stream())
     tdt = torch.float16 if out == 0 else torch.bfloat16
     for step, bits in ((0, 8), (1, 5)):
@@ -158,9 +169,10 @@ def test_gemm_dequant_given_codes(T, out, M, N, K):
 
 
 # ----------------------------------------------------------------------------- whole forward
+@pytest.mark.parametrize("mode", [0] + GEMM_MODES)
 @pytest.mark.parametrize("n,K,N,M", [(64, 1152, 1152, 256), (64, 1152, 3456, 300), (128, 2240, 6720, 130),
                                      (64, 4608, 1152, 77), (128, 5600, 2240, 513), (64, 64, 8, 1)])
-def test_forward_matches_oracle(T, n, K, N, M):
+def test_forward_matches_oracle(T, n, K, N, M, mode):
     rng = np.random.default_rng(n + K + N + M)
     Kp = oracle.padded_k(K, n)
     x = _acts(rng, M, K)
@@ -168,6 +180,7 @@ def test_forward_matches_oracle(T, n, K, N, M):
     s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
     bits_per_step = [8, 6, 5, 4, 3]
     ctx = _ctx(T, [(N, K, w, s_w)], len(bits_per_step), n, M + 5)
+    T.tasq_debug_set_gemm_mode(ctx, mode)
     T.tasq_set_schedule(ctx, np.array([bits_per_step], np.uint8), _stream())
     xd = _dev(x)
     ldy = N + (8 - N % 8) % 8 + 16

@@ -69,6 +69,7 @@ def _load():
         "tasq_debug_gemm_s32": [P, P, i64, i32, i32, P, i64, P],
         "tasq_debug_gemm": [P, P, P, i64, i32, i32, P, i64, i32, P],
         "tasq_debug_stuck_wait": [P, P],
+        "tasq_debug_set_gemm_mode": [P, i32],
         "tasq_trace_enable": [P, i32],
         "tasq_linear_forward_noalloc": [P, i64, i64, i32, P, P, i32, i32, i32, P, i64, i32, P, P],
         "tasq_trace_read": [P, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i32),
@@ -205,6 +206,10 @@ def tasq_debug_gemm(ctx: Context, xq, s_x, M: int, layer: int, step: int, y, ldy
                     stream=None) -> None:
     _check(lib.tasq_debug_gemm(ctx, _ptr(xq), _ptr(s_x), int(M), int(layer), int(step), _ptr(y), int(ldy),
                                int(out_dtype), _stream(stream)))
+
+
+def tasq_debug_set_gemm_mode(ctx: Context, mode: int) -> None:
+    _check(lib.tasq_debug_set_gemm_mode(ctx, int(mode)))
 
 
 def tasq_debug_stuck_wait(ctx: Context, stream=None) -> None:

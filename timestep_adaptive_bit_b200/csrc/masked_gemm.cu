@@ -10,7 +10,8 @@
 // de Hardware"). The bit width is read from the device schedule table inside the kernel, so a
 // new step needs no new weights and no different kernel.
 //
-// Design (one persistent CTA per SM, warp-specialised, 448 threads):
+// Design (one persistent CTA per SM, warp-specialised, 448 threads; the pair kernel in
+// masked_gemm_pair.cu shares the roles and the epilogue):
 //   tile            128 output channels x 256 tokens; the weight tile is the MMA's A operand
 //                   (M = 128), the activation-code tile its B operand (N = 256); K advances in
 //                   stages of 128 bytes = four tcgen05.mma.kind::i8 of K = 32.
@@ -31,55 +32,34 @@
 // Every wait is bounded (ptx::wait_bounded); a wait that runs out records a status bit, raises
 // a CTA-wide abort flag, and every role winds down: the producer waits (bounded) for the loads
 // it issued, the MMA thread for its MMAs, then TMEM is freed and the CTA exits.
-#include <cuda_bf16.h>
-#include <cuda_fp16.h>
-
-#include "../../include/tasq.h"
-#include "ptx.cuh"
-#include "tasq_internal.h"
+#include "gemm_common.cuh"
 
 namespace tasq {
 namespace {
 
-constexpr int kTileCh = kGemmTileCh;      // 128
-constexpr int kTileTok = kGemmTileTok;    // 256
-constexpr int kBlockK = kGemmBlockK;      // 128 bytes
-constexpr int kUmmaK = 32;
+using namespace gemm;
+
+constexpr int kTileCh = kGemmTileCh;      // 128 output channels per tile
+constexpr int kTileTok = kGemmTileTok;    // 256 tokens per tile
 constexpr int kABytes = kTileCh * kBlockK;
 constexpr int kBBytes = kTileTok * kBlockK;
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kAccCols = kTileTok;
-constexpr int kAccStages = 2;
-constexpr uint32_t kTmemCols = kAccCols * kAccStages;   // 512: the whole TMEM of the SM
-constexpr int kEpiWarps = 8;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kMaskWarp0 = 10;
-constexpr int kMaskWarps = 4;
-constexpr int kThreads = 32 * (kEpiWarps + 2 + kMaskWarps);
-constexpr int kMaskThreads = 32 * kMaskWarps;
-constexpr int kEpiThreads = 32 * kEpiWarps;
-constexpr int kEpiCols = kTileTok / (kEpiWarps / 4);     // 128 tokens per epilogue warp
-constexpr int kSxBytesPerWarp = kEpiCols * 4;
+static_assert(kTileTok == kAccCols, "accumulator width");
 
 // Shared-memory plan of one instantiation: stages of (weights, codes), the epilogue's output
-// staging (one 32 x 32 tile per warp), its s_x slices, the barriers.
+// staging (one 32 x 32 box per warp), its s_x slices, the barriers.
 template <int OUT>
 struct Plan {
-  static constexpr int kOutBytes = OUT == static_cast<int>(OutKind::S32) ? 4 : 2;
-  static constexpr int kStages = OUT == static_cast<int>(OutKind::S32) ? 3 : 4;
-  static constexpr int kEpiStageBytes = 32 * 32 * kOutBytes;
+  static constexpr int kStages = OutTraits<OUT>::kS32 ? 3 : 4;
   static constexpr int kEpiOffset = kStages * kStageBytes;
-  static constexpr int kSxOffset = kEpiOffset + kEpiWarps * kEpiStageBytes;
+  static constexpr int kSxOffset = kEpiOffset + kEpiWarps * OutTraits<OUT>::kStageBytes;
   static constexpr int kBarOffset = kSxOffset + kEpiWarps * kSxBytesPerWarp;
   static constexpr int kNumBars = 3 * kStages + 2 * kAccStages + 1;
   static constexpr int kSmemBytes = 1024 /* alignment slack */ + kBarOffset + kNumBars * 8 + 16;
-  static_assert(kSmemBytes <= 232448, "shared memory");
+  static_assert(kSmemBytes <= kMaxSmem, "shared memory");
 };
 
 static_assert(kABytes % (16 * kMaskThreads) == 0, "mask pass must tile the weight stage");
-static_assert(kTileTok % 16 == 0 && kTileTok <= 256, "UMMA N");
-static_assert(kBlockK % kUmmaK == 0, "stage K");
 
 template <int STAGES>
 struct Bars {
@@ -92,29 +72,12 @@ struct Bars {
   __device__ uint32_t drain() const { return base + 8u * (3 * STAGES + 2 * kAccStages); }
 };
 
-__device__ __forceinline__ void raise_failure(uint32_t* status, volatile int* abort_flag, uint32_t bit) {
-  atomicOr(status, bit);
-  *abort_flag = 1;
-}
-
-// y = (acc * s_x) * s_w, each product rounded once in FP32, then rounded to the output type.
-template <int OUT>
-__device__ __forceinline__ uint16_t out_bits(uint32_t acc, float sx, float sw) {
-  const float v = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(acc)), sx), sw);
-  if constexpr (OUT == static_cast<int>(OutKind::F16)) {
-    return __half_as_ushort(__float2half_rn(v));
-  } else {
-    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
-  }
-}
-
 template <int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     masked_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                        const __grid_constant__ CUtensorMap tmap_y, const GemmArgs g) {
   using P = Plan<OUT>;
   constexpr int kStages = P::kStages;
-  constexpr bool kS32 = OUT == static_cast<int>(OutKind::S32);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_addr(smem);
@@ -124,6 +87,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // the next kernel of the stream may be scheduled; it waits for this one before reading
+  ptx::grid_dep_launch_dependents();
 
   // schedule lookup: the step's bit width for this layer
   int bits = g.bits_table[g.bits_index];
@@ -138,12 +103,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(bars.full(s), 1);
-      ptx::mbar_init(bars.masked(s), kMaskThreads);
+      ptx::mbar_init(bars.masked(s), kMaskWarps);
       ptx::mbar_init(bars.empty(s), 1);
     }
     for (int i = 0; i < kAccStages; ++i) {
       ptx::mbar_init(bars.acc_full(i), 1);
-      ptx::mbar_init(bars.acc_empty(i), kEpiThreads);
+      ptx::mbar_init(bars.acc_empty(i), kEpiWarps);
     }
     ptx::mbar_init(bars.drain(), 1);
     *abort_flag = 0;
@@ -173,6 +138,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------------------ TMA producer
       uint32_t s = 0, ph = 0, issued = 0, issued_par = 0;
       bool ok = true;
+      // the activation codes come from the prologue kernel just before this one
+      ptx::grid_dep_wait();
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int mt = tile % g.num_m_tiles;
         const int nt = tile / g.num_m_tiles;
@@ -262,18 +229,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          uint4* wt = reinterpret_cast<uint4*>(smem + s * kABytes);
-#pragma unroll
-          for (int i = 0; i < kABytes / 16 / kMaskThreads; ++i) {
-            uint4 w = wt[i * kMaskThreads + t];
-            w.x &= mask32;
-            w.y &= mask32;
-            w.z &= mask32;
-            w.w &= mask32;
-            wt[i * kMaskThreads + t] = w;
-          }
+          mask_stage<kABytes>(smem + s * kABytes, t, mask32);
           ptx::fence_proxy_async_smem();
-          ptx::mbar_arrive(bars.masked(s));
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(bars.masked(s));
           if (++s == kStages) {
             s = 0;
             ph ^= 1u;
@@ -283,103 +242,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------------------------- epilogue warps
-    const int q = warp & 3;         // TMEM lanes 32 q .. 32 q + 31: channels of this warp
-    const int h = warp >> 2;        // accumulator columns 128 h .. 128 h + 127: tokens
-    uint8_t* stage = smem + P::kEpiOffset + warp * P::kEpiStageBytes;
-    const uint32_t stage_addr = ptx::smem_addr(stage);
-    float* sx_slice = reinterpret_cast<float*>(smem + P::kSxOffset + warp * kSxBytesPerWarp);
-    uint32_t as = 0, aph = 0;
-    bool store_pending = false;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int mt = tile % g.num_m_tiles;
-      const int nt = tile / g.num_m_tiles;
-      const int tok0 = mt * kTileTok + h * kEpiCols;
-      const bool got = ptx::wait_bounded(bars.acc_full(as), aph, limit, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) {
-        if (lane == 0) raise_failure(g.status, abort_flag, TASQ_DEVICE_TIMEOUT_EPILOGUE);
-        break;
-      }
-      ptx::tc_fence_after_sync();
-      const int ch = nt * kTileCh + q * 32 + lane;
-      float sw = 0.0f;
-      if constexpr (!kS32) {
-        if (ch < g.N) sw = g.s_w[ch];
-        // this warp's 128 token scales, read once per tile into its private slice
-        float4 v4;
-        const int m = tok0 + 4 * lane;
-        v4.x = m < g.M ? g.s_x[m] : 0.0f;
-        v4.y = m + 1 < g.M ? g.s_x[m + 1] : 0.0f;
-        v4.z = m + 2 < g.M ? g.s_x[m + 2] : 0.0f;
-        v4.w = m + 3 < g.M ? g.s_x[m + 3] : 0.0f;
-        reinterpret_cast<float4*>(sx_slice)[lane] = v4;
-        __syncwarp();
-      }
-      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + as * kAccCols + h * kEpiCols;
-#pragma unroll 1
-      for (int j = 0; j < kEpiCols / 32; ++j) {
-        uint32_t r[32];
-        ptx::tmem_ld_32x32b_x32(tacc + j * 32, r);
-        ptx::tmem_ld_wait(r);
-        if (j == kEpiCols / 32 - 1) {
-          // the accumulator has been read: hand it back to the MMA before storing
-          ptx::tc_fence_before_sync();
-          ptx::mbar_arrive(bars.acc_empty(as));
-        }
-        const int t0 = tok0 + j * 32;
-        const int c0 = nt * kTileCh + q * 32;
-        // boxes wholly past the last token or channel have nothing to store (warp-uniform)
-        if (t0 >= g.M || c0 >= g.N) continue;
-        const float4* sx4 = reinterpret_cast<const float4*>(sx_slice + j * 32);
-        if (c0 + 32 > g.N && (g.N * P::kOutBytes) % 16 != 0) {
-          // a TMA store writes whole 16-byte granules, so a box whose right edge is not 16-byte
-          // aligned would write past column N: store this one with plain predicated stores
-          const int chl = c0 + lane;
-#pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            const float sxv = kS32 ? 0.0f : sx_slice[j * 32 + t];
-            if (chl < g.N && t0 + t < g.M) {
-              const int64_t idx = static_cast<int64_t>(t0 + t) * g.ldy + chl;
-              if constexpr (kS32) {
-                static_cast<int32_t*>(g.y)[idx] = static_cast<int32_t>(r[t]);
-              } else {
-                const uint16_t b = out_bits<OUT>(r[t], sxv, sw);
-                static_cast<uint16_t*>(g.y)[idx] = b;
-              }
-            }
-          }
-          continue;
-        }
-        if (store_pending) {
-          // the previous bulk store of this warp must have finished reading the staging tile
-          if (lane == 0) ptx::bulk_wait_read0();
-          __syncwarp();
-        }
-        if constexpr (kS32) {
-          uint32_t* st = reinterpret_cast<uint32_t*>(stage);
-#pragma unroll
-          for (int t = 0; t < 32; ++t) st[t * 32 + lane] = r[t];
-        } else {
-          uint16_t* st = reinterpret_cast<uint16_t*>(stage);
-#pragma unroll
-          for (int t4 = 0; t4 < 8; ++t4) {
-            const float4 sx = sx4[t4];
-            const float sxv[4] = {sx.x, sx.y, sx.z, sx.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) st[(4 * t4 + i) * 32 + lane] = out_bits<OUT>(r[4 * t4 + i], sxv[i], sw);
-          }
-        }
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          ptx::tma_store_2d(&tmap_y, stage_addr, c0, t0);
-          ptx::bulk_commit();
-        }
-        store_pending = true;
-      }
-      as ^= 1u;
-      if (as == 0) aph ^= 1u;
-    }
-    if (lane == 0) ptx::bulk_wait0();
+    epilogue_role<OUT, false>(g, &tmap_y, tmem_base, smem + P::kEpiOffset + warp * OutTraits<OUT>::kStageBytes,
+                              reinterpret_cast<float*>(smem + P::kSxOffset + warp * kSxBytesPerWarp), warp, lane,
+                              blockIdx.x, gridDim.x, num_tiles, kTileCh, 0, bars.acc_full(0), bars.acc_empty(0),
+                              limit, abort_flag);
   }
 
   __syncwarp();
@@ -407,8 +273,17 @@ cudaError_t launch_out(const CUtensorMap& tw, const CUtensorMap& tx, const CUten
   }
   const int tiles = g.num_m_tiles * g.num_n_tiles;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  masked_gemm_kernel<OUT><<<grid, kThreads, Plan<OUT>::kSmemBytes, stream>>>(tw, tx, ty, g);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Plan<OUT>::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = use_pdl() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, masked_gemm_kernel<OUT>, tw, tx, ty, g);
 }
 
 __global__ void stuck_wait_kernel(uint32_t* status, uint64_t limit_ns) {

@@ -104,6 +104,10 @@ __global__ void __launch_bounds__(kMaxThreads) prologue_kernel(const PrologueArg
   const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + r_local;
   const bool active = r_local < rows_per_cta && row < a.M;
 
+  // x may be the previous kernel's output: wait for it, then let the GEMM start its setup
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
   __shared__ unsigned int row_max[kMaxRowsPerCta];
   if (tid < rows_per_cta) row_max[tid] = 0u;
   __syncthreads();
@@ -234,15 +238,21 @@ cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
   if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
   const bool vec32 = (reinterpret_cast<uintptr_t>(a.x) % 32 == 0) && (a.ldx % 16 == 0) &&
                      (reinterpret_cast<uintptr_t>(a.xq) % 32 == 0);
-  const unsigned gx = static_cast<unsigned>(grid);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = use_pdl() ? 1 : 0;
   if (a.n == 64) {
-    if (vec32) prologue_kernel<2, true><<<gx, threads, 0, stream>>>(a, R);
-    else prologue_kernel<2, false><<<gx, threads, 0, stream>>>(a, R);
-  } else {
-    if (vec32) prologue_kernel<4, true><<<gx, threads, 0, stream>>>(a, R);
-    else prologue_kernel<4, false><<<gx, threads, 0, stream>>>(a, R);
+    if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<2, true>, a, R);
+    return cudaLaunchKernelEx(&cfg, prologue_kernel<2, false>, a, R);
   }
-  return cudaGetLastError();
+  if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<4, true>, a, R);
+  return cudaLaunchKernelEx(&cfg, prologue_kernel<4, false>, a, R);
 }
 
 }  // namespace tasq

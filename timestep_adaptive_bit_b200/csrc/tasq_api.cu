@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -32,6 +33,14 @@ tasq_status fail_cuda(cudaError_t e, const char* what) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool use_pdl() {
+  static const bool on = [] {
+    const char* v = std::getenv("TASQ_PDL");
+    return v == nullptr || std::string(v) != "0";
+  }();
+  return on;
+}
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -123,6 +132,7 @@ struct tasq_ctx {
   uint32_t* d_status = nullptr;
   uint64_t wait_limit_ns = 1000000000ull;
   float sx_factor = 0.0f;
+  int32_t gemm_mode = 0;   // 0 automatic, 1 one CTA per tile, 2 CTA pairs
   // trace
   int32_t trace_cap = 0, trace_count = 0;
   std::vector<TraceRec> trace;
@@ -206,12 +216,27 @@ tasq_status run_prologue(tasq_ctx* c, const LayerInfo& L, const void* x, int64_t
   return TASQ_OK;
 }
 
+// Which GEMM kernel finishes first: both are persistent, so the time is the number of waves of
+// tiles times the time of one tile. A CTA pair does a 256 x 256 tile on two SMs at about 1.1x the
+// per-SM rate of one CTA on a 128 x 256 tile (measured on B200 at large K); ragged edges and
+// partial last waves decide the rest.
+bool prefer_pair(int64_t M, int64_t N, int num_sms) {
+  const int64_t t1 = ((M + 255) / 256) * ((N + 127) / 128);
+  const int64_t t2 = ((M + 255) / 256) * ((N + 255) / 256);
+  const int64_t slots1 = num_sms, slots2 = num_sms / 2;
+  const double w1 = static_cast<double>((t1 + slots1 - 1) / slots1);
+  const double w2 = static_cast<double>((t2 + slots2 - 1) / slots2);
+  // per-SM work per wave: 128 x 256 for one CTA, 256 x 256 / 2 for a pair
+  return w2 / 1.1 < w1;
+}
+
 tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq, const float* sx, int64_t M,
                      void* y, int64_t ldy, tasq::OutKind out, cudaStream_t s) {
   const LayerInfo& L = c->layers[layer];
+  const bool pair = c->gemm_mode == 2 || (c->gemm_mode == 0 && prefer_pair(M, L.N, c->num_sms));
   CUtensorMap tx;
   tasq_status st = make_tmap_u8(&tx, xq, static_cast<uint64_t>(L.Kp), static_cast<uint64_t>(M), tasq::kGemmBlockK,
-                                tasq::kGemmTileTok);
+                                pair ? tasq::kGemmPairHalf : tasq::kGemmTileTok);
   if (st != TASQ_OK) return st;
   CUtensorMap ty;
   const CUtensorMapDataType dt = out == tasq::OutKind::S32    ? CU_TENSOR_MAP_DATA_TYPE_INT32
@@ -224,8 +249,10 @@ tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq,
   g.M = static_cast<int32_t>(M);
   g.N = L.N;
   g.num_kb = (L.Kp + tasq::kGemmBlockK - 1) / tasq::kGemmBlockK;
-  g.num_m_tiles = static_cast<int32_t>((M + tasq::kGemmTileTok - 1) / tasq::kGemmTileTok);
-  g.num_n_tiles = (L.N + tasq::kGemmTileCh - 1) / tasq::kGemmTileCh;
+  const int tile_tok = pair ? tasq::kGemmPairTile : tasq::kGemmTileTok;
+  const int tile_ch = pair ? tasq::kGemmPairTile : tasq::kGemmTileCh;
+  g.num_m_tiles = static_cast<int32_t>((M + tile_tok - 1) / tile_tok);
+  g.num_n_tiles = (L.N + tile_ch - 1) / tile_ch;
   g.bits_table = c->d_bits;
   g.bits_index = layer * c->num_steps + step;
   g.s_x = sx;
@@ -234,7 +261,8 @@ tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq,
   g.ldy = ldy;
   g.status = c->d_status;
   g.wait_limit_ns = c->wait_limit_ns;
-  cudaError_t e = tasq::launch_masked_gemm(c->tmap_w[layer], tx, ty, g, out, c->num_sms, s);
+  cudaError_t e = pair ? tasq::launch_masked_gemm_pair(c->tmap_w[layer], tx, ty, g, out, c->num_sms, s)
+                       : tasq::launch_masked_gemm(c->tmap_w[layer], tx, ty, g, out, c->num_sms, s);
   if (e != cudaSuccess) return fail_cuda(e, "masked GEMM launch");
   return TASQ_OK;
 }
@@ -484,6 +512,14 @@ tasq_status tasq_debug_gemm(tasq_ctx* c, const int8_t* xq, const float* s_x, int
   if (M == 0) return TASQ_OK;
   const tasq::OutKind out = out_dtype == TASQ_OUT_BF16 ? tasq::OutKind::BF16 : tasq::OutKind::F16;
   return run_gemm(c, layer, step, xq, s_x, M, y, ldy, out, static_cast<cudaStream_t>(stream));
+}
+
+tasq_status tasq_debug_set_gemm_mode(tasq_ctx* c, int32_t mode) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  if (mode < 0 || mode > 2) return fail(TASQ_ERR_INVALID_ARG, "mode must be 0, 1 or 2");
+  c->gemm_mode = mode;
+  return TASQ_OK;
 }
 
 tasq_status tasq_debug_stuck_wait(tasq_ctx* c, void* stream) {

@@ -46,6 +46,13 @@ struct GemmArgs {
 cudaError_t launch_masked_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const CUtensorMap& tmap_y,
                                const GemmArgs& g, OutKind out, int num_sms, cudaStream_t stream);
 
+// The same GEMM over CTA pairs (tcgen05 cta_group::2): tiles of 256 channels x 256 tokens, each
+// CTA holding 128 rows of each operand (tensor-map boxes of 128 x 128 bytes for both).
+cudaError_t launch_masked_gemm_pair(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const CUtensorMap& tmap_y,
+                                    const GemmArgs& g, OutKind out, int num_sms, cudaStream_t stream);
+constexpr int kGemmPairTile = 256;  // channels and tokens per pair tile
+constexpr int kGemmPairHalf = 128;  // operand rows per CTA of a pair
+
 // Geometry of the GEMM tiles (for the host's tensor maps).
 constexpr int kGemmTileCh = 128;    // weight rows per tile
 constexpr int kGemmTileTok = 256;   // activation rows per tile
@@ -53,6 +60,10 @@ constexpr int kGemmBlockK = 128;    // K bytes per pipeline stage
 constexpr int kGemmStoreBox = 32;   // outputs leave in 32 x 32 TMA store boxes
 
 cudaError_t launch_stuck_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
+
+// Whether kernels are launched with programmatic dependent launch, so that a kernel's setup
+// overlaps the tail of the previous kernel on the stream (environment TASQ_PDL=0 turns it off).
+bool use_pdl();
 
 // Host helpers shared by the entry points (defined in tasq_api.cu).
 extern thread_local std::string g_last_error;
