@@ -16,8 +16,8 @@
 // The 32 values sit in 16 register pairs, pair p = (z_p, z_(p+16)), so the butterfly stages with
 // stride 1, 2, 4, 8 are packed FP32x2 add / fma (two independent IEEE round-to-nearest operations
 // each), the stride-16 stage runs inside each pair, and the stride-32 (and, for n = 128,
-// stride-64) stage pairs lane i with lane i ^ 1 (and i ^ 2) through xor shuffles. The stages run
-// in increasing stride, each butterfly (a, b) -> (a + b, a - b) rounded once in FP32, so the codes
+// stride-64) stage pairs lane i with lane i ^ 1 (and i ^ 2) through xor shuffles and one packed
+// fma by +-1 (exact product, one rounding). The stages run in increasing stride, each butterfly (a, b) -> (a + b, a - b) rounded once in FP32, so the codes
 // are the same bits as a textbook FP32 fast Walsh-Hadamard transform produces.
 // The per-row absmax is combined through a shared-memory atomicMax on the float bits (all values
 // are non-negative). No FMA contraction happens anywhere on the path.
@@ -83,15 +83,28 @@ __device__ __forceinline__ float2 mul2(float2 a, float s) {
   return *reinterpret_cast<const float2*>(&r);
 }
 
+// Four INT32 codes to four signed bytes (a in the lowest byte), saturating to [-128, 127].
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
-  const uint32_t lo = __byte_perm(static_cast<uint32_t>(a), static_cast<uint32_t>(b), 0x0040);
-  const uint32_t hi = __byte_perm(static_cast<uint32_t>(c), static_cast<uint32_t>(d), 0x0040);
-  return __byte_perm(lo, hi, 0x5410);
+  uint32_t hi, out;
+  asm("cvt.pack.sat.s8.s32.b32 %0, %2, %1, 0;" : "=r"(hi) : "r"(c), "r"(d));
+  asm("cvt.pack.sat.s8.s32.b32 %0, %2, %1, %3;" : "=r"(out) : "r"(a), "r"(b), "r"(hi));
+  return out;
 }
 
-__device__ __forceinline__ int code(float t) {
-  int q = __float2int_rn(t);
-  return max(-127, min(127, q));
+// RNE code of t = z * fp32(127 / a). With |z| <= a the two roundings keep |t| <= 127 (1 + 2^-23)
+// < 127.5, so the code is always in [-127, 127]; the saturating pack is never reached.
+__device__ __forceinline__ int code(float t) { return __float2int_rn(t); }
+
+// other + s * mine on FP32 pairs with one rounding: s = +1 gives RN(mine + other), s = -1 gives
+// RN(other - mine), the two outputs of a butterfly whose partner value sits in another lane.
+__device__ __forceinline__ float2 fma2_sign(float2 mine, float s, float2 other) {
+  const float2 ss = make_float2(s, s);
+  const uint64_t um = *reinterpret_cast<const uint64_t*>(&mine);
+  const uint64_t us = *reinterpret_cast<const uint64_t*>(&ss);
+  const uint64_t uo = *reinterpret_cast<const uint64_t*>(&other);
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(um), "l"(us), "l"(uo));
+  return *reinterpret_cast<const float2*>(&r);
 }
 
 // LANES = n / 32 lanes per Hadamard block; VEC32: row starts of x and xq are 32-byte aligned.
@@ -168,16 +181,17 @@ __global__ void __launch_bounds__(kMaxThreads) prologue_kernel(const PrologueArg
     v[p].x = __fadd_rn(lo, hi);
     v[p].y = __fsub_rn(lo, hi);
   }
-  // strides 32 (and 64): the partner segment of the block sits in lane ^ m
+  // strides 32 (and 64): the partner segment of the block sits in lane ^ m; the lower lane keeps
+  // mine + other, the upper lane other - mine
 #pragma unroll
   for (int m = 1; m < LANES; m <<= 1) {
-    const bool upper = (seg & m) != 0;
+    const float sgn = (seg & m) != 0 ? -1.0f : 1.0f;
 #pragma unroll
     for (int p = 0; p < 16; ++p) {
-      const float ox = __shfl_xor_sync(0xffffffffu, v[p].x, m);
-      const float oy = __shfl_xor_sync(0xffffffffu, v[p].y, m);
-      v[p].x = upper ? __fsub_rn(ox, v[p].x) : __fadd_rn(v[p].x, ox);
-      v[p].y = upper ? __fsub_rn(oy, v[p].y) : __fadd_rn(v[p].y, oy);
+      float2 o;
+      o.x = __shfl_xor_sync(0xffffffffu, v[p].x, m);
+      o.y = __shfl_xor_sync(0xffffffffu, v[p].y, m);
+      v[p] = fma2_sign(v[p], sgn, o);
     }
   }
 
