@@ -65,6 +65,29 @@ def parse_args(argv=None):
 
 
 # ------------------------------------------------------------------------------ peaks, clocks
+GEMM_SOURCES = ("masked_gemm.cu", "masked_gemm_pair.cu", "gemm_common.cuh", "ptx.cuh")
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per GEMM launch from the committed ncu summary of this workload's step, if the
+    GEMM kernel sources are still the ones the counters were taken on (else None)."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", f"launches_{workload}_step.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_t = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
+    m_h = re.search(r"kernel_sources_sha256:\s*([0-9a-f]{64})", text)
+    if not (m_t and m_h):
+        return None
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "timestep_adaptive_bit_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return int(m_t.group(1)) if h.hexdigest() == m_h.group(1) else None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -427,7 +450,9 @@ def main(argv=None):
         "mean_bits": mean_bits,
         "bitops_saved_modelled": 1.0 - mean_bits / 8.0,
         "roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": int8_burst, "unit": "TFLOP/s",
-                     "frac": (gemm_tops / int8_burst) if gemm_tops else None, "traffic": None,
+                     "frac": (gemm_tops / int8_burst) if gemm_tops else None,
+                     "traffic": profiled_traffic(wl.name),
+                     "traffic_source": f"profiles/launches_{wl.name}_step.md (null once the GEMM sources change)",
                      "kernel": "masked_gemm_kernel", "peak_kind": f"INT8 = 2 x {peak_kind} BF16 burst",
                      "frac_of_sustained": (gemm_tops / int8_sust) if gemm_tops else None},
         "prologue_roofline": {"bound": "hbm", "achieved": pro_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
