@@ -41,21 +41,41 @@ __device__ __forceinline__ void raise_failure(uint32_t* status, volatile int* ab
   *abort_flag = 1;
 }
 
-// y = (acc * s_x) * s_w, each product rounded once in FP32, then rounded to the output type.
+// Packed FP32x2 product, each lane rounded once to nearest even.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  const uint64_t ua = *reinterpret_cast<const uint64_t*>(&a);
+  const uint64_t ub = *reinterpret_cast<const uint64_t*>(&b);
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(ua), "l"(ub));
+  return *reinterpret_cast<const float2*>(&r);
+}
+
+// Two adjacent tokens of one channel: y = (acc * s_x) * s_w in FP32, then a packed FP16 / BF16
+// pair (first token in the low half).
 template <int OUT>
-__device__ __forceinline__ uint16_t out_bits(uint32_t acc, float sx, float sw) {
-  const float v = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(acc)), sx), sw);
+__device__ __forceinline__ uint32_t out_pair(uint32_t a0, uint32_t a1, float2 sx, float sw) {
+  const float2 acc = make_float2(static_cast<float>(static_cast<int32_t>(a0)),
+                                 static_cast<float>(static_cast<int32_t>(a1)));
+  const float2 v = mul2(mul2(acc, sx), make_float2(sw, sw));
   if constexpr (OUT == static_cast<int>(OutKind::F16)) {
-    return __half_as_ushort(__float2half_rn(v));
+    const __half2 h = __floats2half2_rn(v.x, v.y);
+    return *reinterpret_cast<const uint32_t*>(&h);
   } else {
-    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+    return *reinterpret_cast<const uint32_t*>(&h);
   }
 }
 
-// Epilogue role of warps 0..7. Warp w reads TMEM lanes 32 (w % 4) .. +31 (its 32 output channels)
-// and accumulator columns 128 (w / 4) .. +127 (its 128 tokens) in chunks of 32 columns, scales,
-// converts, writes the 32 x 32 box into its private staging buffer in output row order and
-// stores it with one TMA bulk store. Warps never wait on each other.
+// Epilogue role of warps 0..7. Warp w owns TMEM lanes 32 (w % 4) .. +31 (32 output channels) and
+// accumulator columns 128 (w / 4) .. +127 (128 tokens), taken in chunks of 32 columns. Each chunk
+// is scaled, converted and written into the warp's private 32 x 32 staging box in output row
+// order, then stored with one TMA bulk store. Warps never wait on each other.
+//   FP16 / BF16: two 16 x 256-bit TMEM loads give each lane two adjacent tokens of four channels;
+//   the packed pairs are exactly 8 x 8 matrix fragments (row = channel, column = token), which
+//   stmatrix.trans writes token-major into the box, 16 bytes per row, through a 64-byte swizzle
+//   (chunk ^= (row >> 1) & 3) that keeps the eight rows of each matrix on distinct banks; the TMA
+//   store undoes the swizzle.
+//   INT32 (test hook): 32 x 32-bit TMEM loads, one value per lane per store, no swizzle.
 //   ch_per_tile / ch_offset : output channels of tile nt start at nt * ch_per_tile + ch_offset.
 //   acc_full + 8 i          : local barrier the MMA side arrives on when accumulator i is ready.
 //   acc_empty + 8 i         : barrier (local, or in another CTA of the cluster when CLUSTER) that
@@ -84,83 +104,146 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
       break;
     }
     ptx::tc_fence_after_sync();
-    const int c0 = nt * ch_per_tile + ch_offset + q * 32;
-    const int ch = c0 + lane;
-    float sw = 0.0f;
-    if constexpr (!O::kS32) {
-      if (ch < g.N) sw = g.s_w[ch];
-      // this warp's 128 token scales, read once per tile into its private slice
-      float4 v4;
-      const int m = tok0 + 4 * lane;
-      v4.x = m < g.M ? g.s_x[m] : 0.0f;
-      v4.y = m + 1 < g.M ? g.s_x[m + 1] : 0.0f;
-      v4.z = m + 2 < g.M ? g.s_x[m + 2] : 0.0f;
-      v4.w = m + 3 < g.M ? g.s_x[m + 3] : 0.0f;
-      reinterpret_cast<float4*>(sx_slice)[lane] = v4;
-      __syncwarp();
-    }
+    const int c0 = nt * ch_per_tile + ch_offset + q * 32;   // first channel of this warp
     const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + as * kAccCols + h * kEpiCols;
+    if constexpr (O::kS32) {
+      const int ch = c0 + lane;
 #pragma unroll 1
-    for (int j = 0; j < kEpiCols / 32; ++j) {
-      uint32_t r[32];
-      ptx::tmem_ld_32x32b_x32(tacc + j * 32, r);
-      ptx::tmem_ld_wait(r);
-      if (j == kEpiCols / 32 - 1) {
-        // the accumulator has been read: hand it back to the MMA before storing (one arrival
-        // per warp, after every lane's TMEM reads are ordered before the warp barrier)
-        ptx::tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) {
-          if constexpr (CLUSTER) ptx::mbar_arrive_cluster(acc_empty + 8u * as);
-          else ptx::mbar_arrive(acc_empty + 8u * as);
-        }
-      }
-      const int t0 = tok0 + j * 32;
-      // boxes wholly past the last token or channel have nothing to store (warp-uniform)
-      if (t0 >= g.M || c0 >= g.N) continue;
-      if (c0 + 32 > g.N && (g.N * O::kBytes) % 16 != 0) {
-        // a TMA store writes whole 16-byte granules, so a box whose right edge is not 16-byte
-        // aligned would write past column N: store this one with plain predicated stores
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          if (ch < g.N && t0 + t < g.M) {
-            const int64_t idx = static_cast<int64_t>(t0 + t) * g.ldy + ch;
-            if constexpr (O::kS32) {
-              static_cast<int32_t*>(g.y)[idx] = static_cast<int32_t>(r[t]);
-            } else {
-              static_cast<uint16_t*>(g.y)[idx] = out_bits<OUT>(r[t], sx_slice[j * 32 + t], sw);
-            }
+      for (int j = 0; j < kEpiCols / 32; ++j) {
+        uint32_t r[32];
+        ptx::tmem_ld_32x32b_x32(tacc + j * 32, r);
+        ptx::tmem_ld_wait(r);
+        if (j == kEpiCols / 32 - 1) {
+          ptx::tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (CLUSTER) ptx::mbar_arrive_cluster(acc_empty + 8u * as);
+            else ptx::mbar_arrive(acc_empty + 8u * as);
           }
         }
-        continue;
-      }
-      if (store_pending) {
-        // the previous bulk store of this warp must have finished reading the staging tile
-        if (lane == 0) ptx::bulk_wait_read0();
-        __syncwarp();
-      }
-      if constexpr (O::kS32) {
+        const int t0 = tok0 + j * 32;
+        if (t0 >= g.M || c0 >= g.N) continue;
+        if (c0 + 32 > g.N && (g.N * O::kBytes) % 16 != 0) {
+          // a TMA store writes whole 16-byte granules, so a box whose right edge is not 16-byte
+          // aligned would write past column N: store this one with plain predicated stores
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            if (ch < g.N && t0 + t < g.M)
+              static_cast<int32_t*>(g.y)[static_cast<int64_t>(t0 + t) * g.ldy + ch] = static_cast<int32_t>(r[t]);
+          }
+          continue;
+        }
+        if (store_pending) {
+          if (lane == 0) ptx::bulk_wait_read0();
+          __syncwarp();
+        }
         uint32_t* st = reinterpret_cast<uint32_t*>(stage);
 #pragma unroll
         for (int t = 0; t < 32; ++t) st[t * 32 + lane] = r[t];
-      } else {
-        const float4* sx4 = reinterpret_cast<const float4*>(sx_slice + j * 32);
-        uint16_t* st = reinterpret_cast<uint16_t*>(stage);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::tma_store_2d(tmap_y, stage_addr, c0, t0);
+          ptx::bulk_commit();
+        }
+        store_pending = true;
+      }
+    } else {
+      // this lane's four channels: c0 + 16 g + 8 o + lane / 4 for lane half g and octet o
+      float sw[2][2];
 #pragma unroll
-        for (int t4 = 0; t4 < 8; ++t4) {
-          const float4 sx = sx4[t4];
-          const float sxv[4] = {sx.x, sx.y, sx.z, sx.w};
+      for (int gg = 0; gg < 2; ++gg) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) st[(4 * t4 + i) * 32 + lane] = out_bits<OUT>(r[4 * t4 + i], sxv[i], sw);
+        for (int o = 0; o < 2; ++o) {
+          const int ch = c0 + 16 * gg + 8 * o + (lane >> 2);
+          sw[gg][o] = ch < g.N ? g.s_w[ch] : 0.0f;
         }
       }
-      ptx::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        ptx::tma_store_2d(tmap_y, stage_addr, c0, t0);
-        ptx::bulk_commit();
+      // this warp's 128 token scales, read once per tile into its private slice
+      {
+        float4 v4;
+        const int m = tok0 + 4 * lane;
+        v4.x = m < g.M ? g.s_x[m] : 0.0f;
+        v4.y = m + 1 < g.M ? g.s_x[m + 1] : 0.0f;
+        v4.z = m + 2 < g.M ? g.s_x[m + 2] : 0.0f;
+        v4.w = m + 3 < g.M ? g.s_x[m + 3] : 0.0f;
+        reinterpret_cast<float4*>(sx_slice)[lane] = v4;
+        __syncwarp();
       }
-      store_pending = true;
+#pragma unroll 1
+      for (int j = 0; j < kEpiCols / 32; ++j) {
+        uint32_t ra[16], rb[16];   // lanes 32 q + 0 .. 15 and 32 q + 16 .. 31
+        ptx::tmem_ld_16x256b_x4(tacc + j * 32, ra);
+        ptx::tmem_ld_16x256b_x4(tacc + (16u << 16) + j * 32, rb);
+        ptx::tmem_ld_wait(ra, rb);
+        if (j == kEpiCols / 32 - 1) {
+          // the accumulator has been read: hand it back to the MMA before storing (one arrival
+          // per warp, after every lane's TMEM reads are ordered before the warp barrier)
+          ptx::tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (CLUSTER) ptx::mbar_arrive_cluster(acc_empty + 8u * as);
+            else ptx::mbar_arrive(acc_empty + 8u * as);
+          }
+        }
+        const int t0 = tok0 + j * 32;
+        // boxes wholly past the last token or channel have nothing to store (warp-uniform)
+        if (t0 >= g.M || c0 >= g.N) continue;
+        const float* sxc = sx_slice + j * 32;
+        if (c0 + 32 > g.N && (g.N * O::kBytes) % 16 != 0) {
+          // ragged last box whose edge is not 16-byte aligned: plain predicated stores
+#pragma unroll
+          for (int gg = 0; gg < 2; ++gg) {
+            const uint32_t* rr = gg == 0 ? ra : rb;
+#pragma unroll
+            for (int o = 0; o < 2; ++o) {
+              const int ch = c0 + 16 * gg + 8 * o + (lane >> 2);
+#pragma unroll
+              for (int r = 0; r < 4; ++r) {
+                const int tl = 8 * r + 2 * (lane & 3);
+                const uint32_t pr = out_pair<OUT>(rr[4 * r + 2 * o], rr[4 * r + 2 * o + 1],
+                                                  make_float2(sxc[tl], sxc[tl + 1]), sw[gg][o]);
+                if (ch < g.N) {
+                  uint16_t* y = static_cast<uint16_t*>(g.y);
+                  if (t0 + tl < g.M) y[static_cast<int64_t>(t0 + tl) * g.ldy + ch] = static_cast<uint16_t>(pr & 0xFFFFu);
+                  if (t0 + tl + 1 < g.M) y[static_cast<int64_t>(t0 + tl + 1) * g.ldy + ch] = static_cast<uint16_t>(pr >> 16);
+                }
+              }
+            }
+          }
+          continue;
+        }
+        if (store_pending) {
+          // the previous bulk store of this warp must have finished reading the staging box
+          if (lane == 0) ptx::bulk_wait_read0();
+          __syncwarp();
+        }
+        float2 sx2[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) sx2[r] = *reinterpret_cast<const float2*>(sxc + 8 * r + 2 * (lane & 3));
+        // row `lane` of the box is token t0 + lane; its 16-byte chunk c holds channels 8c .. 8c + 7
+        const uint32_t row_addr = stage_addr + 64u * lane;
+        const uint32_t swz = (static_cast<uint32_t>(lane) >> 1) & 3u;
+#pragma unroll
+        for (int gg = 0; gg < 2; ++gg) {
+          const uint32_t* rr = gg == 0 ? ra : rb;
+#pragma unroll
+          for (int o = 0; o < 2; ++o) {
+            uint32_t p[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) p[r] = out_pair<OUT>(rr[4 * r + 2 * o], rr[4 * r + 2 * o + 1], sx2[r], sw[gg][o]);
+            const uint32_t chunk = static_cast<uint32_t>(2 * gg + o);
+            ptx::stmatrix_x4_trans(row_addr + 16u * (chunk ^ swz), p[0], p[1], p[2], p[3]);
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::tma_store_2d(tmap_y, stage_addr, c0, t0);
+          ptx::bulk_commit();
+        }
+        store_pending = true;
+      }
     }
     as ^= 1u;
     if (as == 0) aph ^= 1u;

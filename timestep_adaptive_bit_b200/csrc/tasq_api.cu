@@ -75,7 +75,8 @@ tasq_status make_tmap_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64
 }
 
 // 2-D output tensor [rows, cols] (element type `dt`, row stride `ld` elements) written in
-// boxes of 32 x 32 by TMA stores; elements outside [rows, cols] are never written.
+// boxes of 32 x 32 by TMA stores; elements outside [rows, cols] are never written. 16-bit boxes
+// are read from shared memory with the 64-byte swizzle the epilogue writes them in.
 tasq_status make_tmap_out(CUtensorMap* m, void* base, CUtensorMapDataType dt, uint32_t elem_bytes, uint64_t cols,
                           uint64_t rows, uint64_t ld) {
   auto fn = encode_fn();
@@ -84,7 +85,10 @@ tasq_status make_tmap_out(CUtensorMap* m, void* base, CUtensorMapDataType dt, ui
   const cuuint64_t strides[1] = {ld * elem_bytes};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(tasq::kGemmStoreBox), static_cast<cuuint32_t>(tasq::kGemmStoreBox)};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+  // 16-bit outputs are staged in 64-byte swizzled boxes (32 channels x 2 bytes per row), 32-bit
+  // outputs in plain ones
+  const CUtensorMapSwizzle sw = elem_bytes == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = fn(m, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(TASQ_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed with CUresult " + std::to_string(r));

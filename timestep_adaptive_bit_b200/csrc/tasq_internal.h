@@ -75,7 +75,8 @@ size_t round_up(size_t v, size_t a);
 // UINT8 [rows, cols] tensor (row stride cols bytes) read in 128-byte-swizzled boxes.
 tasq_status make_tmap_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
                          uint32_t box_rows);
-// Output tensor [rows, cols] (row stride ld elements) written in 32 x 32 boxes.
+// Output tensor [rows, cols] (row stride ld elements) written in 32 x 32 boxes (64-byte swizzled
+// staging for 2-byte elements, plain for 4-byte ones).
 tasq_status make_tmap_out(CUtensorMap* m, void* base, CUtensorMapDataType dt, uint32_t elem_bytes, uint64_t cols,
                           uint64_t rows, uint64_t ld);
 
