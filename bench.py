@@ -61,7 +61,22 @@ def parse_args(argv=None):
     p.add_argument("--reps", type=int, default=20)
     p.add_argument("--gemm-mode", type=int, default=0, choices=[0, 1, 2],
                    help="GEMM kernel: 0 automatic, 1 one CTA per tile, 2 CTA pairs")
+    p.add_argument("--mask-mode", type=int, default=0, choices=[0, 1, 2],
+                   help="LSB mask: 0 automatic, 1 inside the GEMM on every tile, 2 once ahead in the prologue launch")
     return p.parse_args(argv)
+
+
+def build_library():
+    """Compile libtasq.so if stale and return the imported package. The build script is loaded
+    by its path: importing the package first would load the library it is about to build."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_tasq_build", os.path.join(ROOT, "timestep_adaptive_bit_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import timestep_adaptive_bit_b200
+    return timestep_adaptive_bit_b200
 
 
 # ------------------------------------------------------------------------------ peaks, clocks
@@ -225,7 +240,7 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------------------ GPU leg
-def setup_workload(T, torch, wl, device, out_dtype):
+def setup_workload(T, torch, wl, device, out_dtype, gemm_mode=0, mask_mode=0):
     """Context with every layer of the workload, one activation buffer per (block, layer),
     one output buffer per distinct N. Weights and activations drawn on the device."""
     L = wl.num_layers
@@ -240,6 +255,8 @@ def setup_workload(T, torch, wl, device, out_dtype):
                                T.TASQ_OUT_F16 if out_dtype == "f16" else T.TASQ_OUT_BF16, stream)
     torch.cuda.synchronize()
     del keep, layers
+    T.tasq_debug_set_gemm_mode(ctx, gemm_mode)
+    T.tasq_debug_set_mask_mode(ctx, mask_mode)
     T.tasq_set_schedule(ctx, workloads.schedule(wl), stream)
     xs = [workloads.activations_torch(wl, l, device) for l in range(L)]
     tdt = torch.float16 if out_dtype == "f16" else torch.bfloat16
@@ -271,6 +288,7 @@ def profile_case(args):
     s = torch.cuda.current_stream()
     ctx = T.tasq_linear_create([(N, K, w, s_w)], 1, wl.hadamard_n, wl.tokens, T.TASQ_OUT_F16, s)
     T.tasq_debug_set_gemm_mode(ctx, args.gemm_mode)
+    T.tasq_debug_set_mask_mode(ctx, args.mask_mode)
     bits = 5 if args.bits is None else args.bits
     T.tasq_set_schedule(ctx, np.array([[bits]], np.uint8), s)
     x = workloads.activations_torch(wl, j, dev)
@@ -298,6 +316,7 @@ def sweep_bits(args):
     s = torch.cuda.current_stream()
     ctx = T.tasq_linear_create([(N, K, w, s_w)], 8, wl.hadamard_n, M, T.TASQ_OUT_F16, s)
     T.tasq_debug_set_gemm_mode(ctx, args.gemm_mode)
+    T.tasq_debug_set_mask_mode(ctx, args.mask_mode)
     T.tasq_set_schedule(ctx, np.array([[8, 7, 6, 5, 4, 3, 2, 1]], np.uint8), s)
     # several input buffers so consecutive launches do not find their activations in L2
     nbuf = max(2, int(math.ceil(3 * 126e6 / (M * K * 2))))
@@ -305,7 +324,7 @@ def sweep_bits(args):
     y = torch.empty((M, N), dtype=torch.float16, device=dev)
     peaks, peak_kind = load_peaks()
     out = {"sweep": f"{name}:{wl.block_layers[j][0]}", "M": M, "K": K, "N": N, "reps": args.reps,
-           "gemm_mode": args.gemm_mode, "bits": {}}
+           "gemm_mode": args.gemm_mode, "mask_mode": args.mask_mode, "bits": {}}
     for step in range(8):
         for r in range(3):
             T.tasq_linear_forward(ctx, xs[r % nbuf], M, K, 0, step, y, N, s)
@@ -319,7 +338,8 @@ def sweep_bits(args):
         out["bits"][8 - step] = {"gemm_us": 1e3 * tr["gemm_ms"] / args.reps, "gemm_tops": g_tops,
                                  "gemm_frac_int8_burst": g_tops / (peaks["bf16_tflops"] * INT8_OVER_BF16),
                                  "prologue_us": 1e3 * tr["prologue_ms"] / args.reps, "prologue_gbs": p_gbs,
-                                 "prologue_frac_hbm": p_gbs / peaks["hbm_gbs"]}
+                                 "prologue_frac_hbm": p_gbs / peaks["hbm_gbs"],
+                                 "forward_us": 1e3 * (tr["prologue_ms"] + tr["gemm_ms"]) / args.reps}
     out["device_status"] = T.tasq_get_device_status(ctx)
     print(json.dumps(out), flush=True)
     return 0 if out["device_status"] == 0 else 1
@@ -337,9 +357,7 @@ def main(argv=None):
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
-    from timestep_adaptive_bit_b200 import build as _build
-    _build.build()
-    import timestep_adaptive_bit_b200 as T
+    T = build_library()
 
     if args.profile_case:
         return profile_case(args)
@@ -352,7 +370,7 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
 
     wl = workloads.WORKLOADS[args.workload]
-    ctx, xs, ys = setup_workload(T, torch, wl, device, args.out_dtype)
+    ctx, xs, ys = setup_workload(T, torch, wl, device, args.out_dtype, args.gemm_mode, args.mask_mode)
     stream = torch.cuda.current_stream()
     L = wl.num_layers
 

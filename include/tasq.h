@@ -80,8 +80,9 @@ typedef struct tasq_ctx tasq_ctx;
 
 /*
  * Create a context owning one shared weight buffer for `num_layers` layers, a device schedule
- * table bits[num_layers][num_steps] (every entry initialised to 8 = full precision), and an
- * activation workspace for up to `max_tokens` tokens.
+ * table bits[num_layers][num_steps] (every entry initialised to 8 = full precision), an
+ * activation workspace for up to `max_tokens` tokens, and a transient buffer for one layer's
+ * masked weights (the largest N x Kp of the layers).
  *   out         : receives the context; *out is set to NULL on failure.
  *   layers      : host array [num_layers] of layer descriptors.
  *   hadamard_n  : block size of the Hadamard transform along K, 64 or 128.
@@ -113,11 +114,14 @@ tasq_status tasq_set_schedule(tasq_ctx* ctx, const uint8_t* bits_host, void* str
  *           (elements, >= N, % 8 == 0).
  * Two kernels run on `stream`: the prologue (block Hadamard of size n along K with zero
  * padding to Kp, per-token absmax, s_x = absmax / (127 sqrt(n)), codes RNE(z * 127 / absmax)
- * in [-127, 127]) into the context workspace, then the GEMM, which reads bits[layer][step]
- * from the device table, clears the low bit planes of each weight tile as it streams into
- * shared memory, accumulates exactly in INT32 and writes y = acc * s_x[m] * s_w[n].
- * Uses the context workspace: forwards of one context must not overlap in time on different
- * streams.
+ * in [-127, 127]) into the context workspace, then the GEMM, which accumulates exactly in INT32
+ * and writes y = acc * s_x[m] * s_w[n]. The weights' low bit planes are cleared according to
+ * bits[layer][step] read from the device table: when the last table given to
+ * tasq_set_schedule drops bits for this (layer, step), the prologue launch writes the masked
+ * layer into the context's masked-weight buffer once and the GEMM reads that; otherwise the
+ * GEMM reads the stored weights and masks each tile in shared memory if the device table asks
+ * for it. Uses the context workspace and masked-weight buffer: forwards of one context must not
+ * overlap in time on different streams.
  */
 tasq_status tasq_linear_forward(tasq_ctx* ctx, const void* x, int64_t M, int64_t ldx, int32_t layer,
                                 int32_t step, void* y, int64_t ldy, void* stream);
@@ -167,9 +171,20 @@ tasq_status tasq_debug_gemm(tasq_ctx* ctx, const int8_t* xq, const float* s_x, i
  * Test hook: which GEMM kernel later forwards of this context use. 0 (default) lets the library
  * choose per launch from the wave count of each kernel's tiles, 1 forces one CTA per 128 x 256
  * tile (tcgen05 cta_group::1), 2 forces CTA pairs on 256 x 256 tiles (tcgen05 cta_group::2).
- * Both compute identical results.
+ * Both compute identical results. Any other mode is TASQ_ERR_INVALID_ARG.
  */
 tasq_status tasq_debug_set_gemm_mode(tasq_ctx* ctx, int32_t mode);
+
+/*
+ * Test hook: where later forwards (and tasq_debug_gemm / tasq_debug_gemm_s32) apply the step's
+ * LSB mask to the weights (TASQ, "LSB masking" of the stored INT8 weights). 0 (default): ahead of
+ * the GEMM, in the prologue launch, into a context-owned copy of the layer's weights whenever the
+ * last schedule given to tasq_set_schedule has bits < 8 for the (layer, step), else inside the
+ * GEMM; 1: always inside the GEMM, on every weight tile it loads; 2: always ahead. Every mode reads
+ * the bit width from the device schedule table, so all give identical results for every table.
+ * Any other mode is TASQ_ERR_INVALID_ARG.
+ */
+tasq_status tasq_debug_set_mask_mode(tasq_ctx* ctx, int32_t mode);
 
 /*
  * Failure-detection hook: launch one CTA that waits, with the context's wait limit, on a

@@ -13,9 +13,8 @@ HEADER = os.path.join(ROOT, "include", "tasq.h")
 
 @pytest.fixture(scope="module")
 def tasq():
-    from timestep_adaptive_bit_b200 import build
-    build.build()
-    import timestep_adaptive_bit_b200 as t
+    from conftest import build_library
+    t = build_library()
     return t
 
 

@@ -28,9 +28,8 @@ ABS_TINY = 2.0 ** -24
 @pytest.fixture(scope="module")
 def T():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
-    from timestep_adaptive_bit_b200 import build
-    build.build()
-    import timestep_adaptive_bit_b200 as t
+    from conftest import build_library
+    t = build_library()
     torch.cuda.init()
     return t
 
@@ -93,14 +92,22 @@ def test_prologue_matches_oracle(T, n, K, M):
 
 
 # ----------------------------------------------------------------------------- GEMM, exact
-# GEMM kernels: 1 = one CTA per 128 x 256 tile, 2 = CTA pairs on 256 x 256 tiles
-GEMM_MODES = [1, 2]
+# (GEMM kernel, mask placement): kernel 1 = one CTA per 128 x 256 tile, 2 = CTA pairs on
+# 256 x 256 tiles; placement 1 = every weight tile masked in shared memory inside the GEMM,
+# 2 = the layer's weights masked once ahead of the GEMM in the prologue launch
+GEMM_MODES = [(1, 1), (1, 2), (2, 1), (2, 2)]
+
+
+def _set_modes(T, ctx, mode):
+    gemm, mask = mode
+    T.tasq_debug_set_gemm_mode(ctx, gemm)
+    T.tasq_debug_set_mask_mode(ctx, mask)
 
 
 @pytest.mark.parametrize("mode", GEMM_MODES)
 @pytest.mark.parametrize("M,N,K,n", [(1, 1, 64, 64), (256, 128, 128, 64), (300, 200, 1152, 64), (513, 384, 192, 64),
                                      (100, 1152, 2240, 128), (257, 130, 4608, 64), (64, 2000, 64, 64),
-                                     (700, 520, 320, 64)])
+                                     (700, 520, 320, 64), (576, 256, 1152, 64)])
 def test_gemm_s32_bit_exact_all_bits(T, M, N, K, n, mode):
     rng = np.random.default_rng(M * 7 + N * 13 + K)
     Kp = oracle.padded_k(K, n)
@@ -108,7 +115,7 @@ def test_gemm_s32_bit_exact_all_bits(T, M, N, K, n, mode):
     q = rng.integers(-127, 128, size=(M, Kp)).astype(np.int8)
     steps = 8
     ctx = _ctx(T, [(N, K, w, np.ones(N, np.float32))], steps, n, M)
-    T.tasq_debug_set_gemm_mode(ctx, mode)
+    _set_modes(T, ctx, mode)
     bits = np.array([[8, 7, 6, 5, 4, 3, 2, 1]], np.uint8)
     T.tasq_set_schedule(ctx, bits, _stream())
     qd = _dev(q)
@@ -133,7 +140,7 @@ def test_gemm_extreme_values(T, mode):
     q = np.full((M, K), -127, np.int8)
     q[::3] = 127
     ctx = _ctx(T, [(N, K, w, np.ones(N, np.float32))], 2, 64, M)
-    T.tasq_debug_set_gemm_mode(ctx, mode)
+    _set_modes(T, ctx, mode)
     T.tasq_set_schedule(ctx, np.array([[8, 1]], np.uint8), _stream())
     acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
     for step, bits in ((0, 8), (1, 1)):
@@ -155,7 +162,7 @@ def test_gemm_dequant_given_codes(T, out, M, N, K, mode):
     s_x = rng.uniform(0.01, 3.0, size=M).astype(np.float32)
     s_x[0] = 0.0
     ctx = _ctx(T, [(N, K, w, s_w)], 2, 64, M)
-    T.tasq_debug_set_gemm_mode(ctx, mode)
+    _set_modes(T, ctx, mode)
     T.tasq_set_schedule(ctx, np.array([[8, 5]], np.uint8), _stream())
     tdt = torch.float16 if out == 0 else torch.bfloat16
     for step, bits in ((0, 8), (1, 5)):
@@ -169,7 +176,7 @@ def test_gemm_dequant_given_codes(T, out, M, N, K, mode):
 
 
 # ----------------------------------------------------------------------------- whole forward
-@pytest.mark.parametrize("mode", [0] + GEMM_MODES)
+@pytest.mark.parametrize("mode", [(0, 0)] + GEMM_MODES)
 @pytest.mark.parametrize("n,K,N,M", [(64, 1152, 1152, 256), (64, 1152, 3456, 300), (128, 2240, 6720, 130),
                                      (64, 4608, 1152, 77), (128, 5600, 2240, 513), (64, 64, 8, 1)])
 def test_forward_matches_oracle(T, n, K, N, M, mode):
@@ -180,7 +187,7 @@ def test_forward_matches_oracle(T, n, K, N, M, mode):
     s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
     bits_per_step = [8, 6, 5, 4, 3]
     ctx = _ctx(T, [(N, K, w, s_w)], len(bits_per_step), n, M + 5)
-    T.tasq_debug_set_gemm_mode(ctx, mode)
+    _set_modes(T, ctx, mode)
     T.tasq_set_schedule(ctx, np.array([bits_per_step], np.uint8), _stream())
     xd = _dev(x)
     ldy = N + (8 - N % 8) % 8 + 16
@@ -224,7 +231,11 @@ def test_schedule_is_stream_ordered(T):
     assert torch.equal(ys[0], ys[2])
 
 
-def test_multi_layer_context_uses_each_layers_weights(T):
+@pytest.mark.parametrize("mask", [0, 1, 2])
+def test_multi_layer_context_uses_each_layers_weights(T, mask):
+    """Every (layer, step) of a 4 x 3 schedule enqueued back to back on one stream before a single
+    synchronize: forwards of different layers reuse the context's workspace and masked-weight
+    buffer, so each kernel must wait for the one before it that reads them."""
     rng = np.random.default_rng(9)
     n, M = 64, 200
     shapes = [(1152, 3456), (1152, 1152), (4608, 1152), (64, 200)]
@@ -235,17 +246,24 @@ def test_multi_layer_context_uses_each_layers_weights(T):
         layers.append((N, K, w, s_w))
         xs.append(_acts(rng, M, K))
     ctx = _ctx(T, layers, 3, n, M)
+    T.tasq_debug_set_mask_mode(ctx, mask)
     sched = np.array([[8, 4, 6], [5, 8, 2], [7, 7, 1], [1, 2, 3]], np.uint8)
     T.tasq_set_schedule(ctx, sched, _stream())
-    for layer, ((N, K, w, s_w), x) in enumerate(zip(layers, xs)):
-        for step in range(3):
+    xds = [_dev(x) for x in xs]
+    outs = {}
+    for step in range(3):
+        for layer, (N, K, _, _) in enumerate(layers):
             assert T.tasq_layer_info(ctx, layer) == (N, K, K)
             y = torch.empty((M, N), dtype=torch.float16, device="cuda")
-            T.tasq_linear_forward(ctx, _dev(x), M, K, layer, step, y, N, _stream())
-            torch.cuda.synchronize()
-            ref = oracle.masked_linear(x, w, s_w, int(sched[layer, step]), n)["y"]
-            got = y.float().cpu().numpy().astype(np.float64)
-            assert np.all(np.abs(got - ref) <= F16_REL * np.abs(ref) + ABS_TINY), (layer, step)
+            T.tasq_linear_forward(ctx, xds[layer], M, K, layer, step, y, N, _stream())
+            outs[layer, step] = y
+    torch.cuda.synchronize()
+    for (layer, step), y in outs.items():
+        N, K, w, s_w = layers[layer]
+        ref = oracle.masked_linear(xs[layer], w, s_w, int(sched[layer, step]), n)["y"]
+        got = y.float().cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(got - ref) <= F16_REL * np.abs(ref) + ABS_TINY), (layer, step)
+    assert T.tasq_get_device_status(ctx) == 0
 
 
 def test_bf16_forward(T):
@@ -291,6 +309,9 @@ def test_argument_errors_on_device(T):
     assert err(T.tasq_linear_forward, ctx, x, -1, K, 0, 0, y, N, s) == T.TASQ_ERR_INVALID_ARG
     assert err(T.tasq_set_schedule, ctx, np.array([[8, 0]], np.uint8), s) == T.TASQ_ERR_INVALID_ARG
     assert err(T.tasq_set_schedule, ctx, np.array([[9, 8]], np.uint8), s) == T.TASQ_ERR_INVALID_ARG
+    assert err(T.tasq_debug_set_gemm_mode, ctx, 3) == T.TASQ_ERR_INVALID_ARG
+    assert err(T.tasq_debug_set_mask_mode, ctx, 3) == T.TASQ_ERR_INVALID_ARG
+    assert err(T.tasq_debug_set_mask_mode, ctx, -1) == T.TASQ_ERR_INVALID_ARG
     T.tasq_linear_forward(ctx, x, 0, K, 0, 0, y, N, s)        # M = 0: nothing to do
     assert T.tasq_get_device_status(ctx) == 0
     with pytest.raises(T.TasqError):

@@ -21,9 +21,8 @@ ABS_TINY = 2.0 ** -24
 @pytest.fixture(scope="module")
 def T():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
-    from timestep_adaptive_bit_b200 import build
-    build.build()
-    import timestep_adaptive_bit_b200 as t
+    from conftest import build_library
+    t = build_library()
     return t
 
 

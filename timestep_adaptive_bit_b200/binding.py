@@ -52,7 +52,7 @@ class tasq_layer_desc(ctypes.Structure):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m timestep_adaptive_bit_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python timestep_adaptive_bit_b200/build.py` "
             "(or __graft_entry__.build()); there is no fallback implementation")
     lib = ctypes.CDLL(LIB_PATH)
     P = ctypes.c_void_p
@@ -70,6 +70,7 @@ def _load():
         "tasq_debug_gemm": [P, P, P, i64, i32, i32, P, i64, i32, P],
         "tasq_debug_stuck_wait": [P, P],
         "tasq_debug_set_gemm_mode": [P, i32],
+        "tasq_debug_set_mask_mode": [P, i32],
         "tasq_trace_enable": [P, i32],
         "tasq_linear_forward_noalloc": [P, i64, i64, i32, P, P, i32, i32, i32, P, i64, i32, P, P],
         "tasq_trace_read": [P, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i32),
@@ -210,6 +211,10 @@ def tasq_debug_gemm(ctx: Context, xq, s_x, M: int, layer: int, step: int, y, ldy
 
 def tasq_debug_set_gemm_mode(ctx: Context, mode: int) -> None:
     _check(lib.tasq_debug_set_gemm_mode(ctx, int(mode)))
+
+
+def tasq_debug_set_mask_mode(ctx: Context, mode: int) -> None:
+    _check(lib.tasq_debug_set_mask_mode(ctx, int(mode)))
 
 
 def tasq_debug_stuck_wait(ctx: Context, stream=None) -> None:

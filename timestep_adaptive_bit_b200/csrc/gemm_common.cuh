@@ -14,9 +14,9 @@ namespace gemm {
 
 constexpr int kBlockK = kGemmBlockK;          // 128 bytes of K per pipeline stage
 constexpr int kUmmaK = 32;                    // K of one tcgen05.mma.kind::i8
-constexpr int kAccCols = 256;                 // tokens per tile = INT32 TMEM columns per accumulator
+constexpr int kAccCols = 256;                 // widest tile: tokens = INT32 TMEM columns per accumulator
 constexpr int kAccStages = 2;
-constexpr uint32_t kTmemCols = kAccCols * kAccStages;   // 512: the whole TMEM of the SM
+constexpr uint32_t kTmemCols = 512;           // the whole TMEM of the SM
 constexpr int kEpiWarps = 8;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
@@ -25,8 +25,7 @@ constexpr int kMaskWarps = 4;
 constexpr int kThreads = 32 * (kEpiWarps + 2 + kMaskWarps);
 constexpr int kMaskThreads = 32 * kMaskWarps;
 constexpr int kEpiThreads = 32 * kEpiWarps;
-constexpr int kEpiCols = kAccCols / (kEpiWarps / 4);     // 128 tokens per epilogue warp
-constexpr int kSxBytesPerWarp = kEpiCols * 4;
+constexpr int kSxBytesPerWarp = (kAccCols / 2) * 4;      // token scales of one epilogue warp
 constexpr int kMaxSmem = 232448;
 
 template <int OUT>
@@ -66,8 +65,9 @@ __device__ __forceinline__ uint32_t out_pair(uint32_t a0, uint32_t a1, float2 sx
   }
 }
 
-// Epilogue role of warps 0..7. Warp w owns TMEM lanes 32 (w % 4) .. +31 (32 output channels) and
-// accumulator columns 128 (w / 4) .. +127 (128 tokens), taken in chunks of 32 columns. Each chunk
+// Epilogue role of warps 0..7 for tiles of TOK tokens (256 or 192). Warp w owns TMEM lanes
+// 32 (w % 4) .. +31 (32 output channels) and accumulator columns TOK/2 (w / 4) .. +TOK/2 - 1,
+// taken in chunks of 32 columns; accumulator i starts at TMEM column i * TOK. Each chunk
 // is scaled, converted and written into the warp's private 32 x 32 staging box in output row
 // order, then stored with one TMA bulk store. Warps never wait on each other.
 //   FP16 / BF16: two 16 x 256-bit TMEM loads give each lane two adjacent tokens of four channels;
@@ -80,15 +80,17 @@ __device__ __forceinline__ uint32_t out_pair(uint32_t a0, uint32_t a1, float2 sx
 //   acc_full + 8 i          : local barrier the MMA side arrives on when accumulator i is ready.
 //   acc_empty + 8 i         : barrier (local, or in another CTA of the cluster when CLUSTER) that
 //                             each epilogue warp arrives on once, after reading accumulator i.
-template <int OUT, bool CLUSTER>
+template <int OUT, bool CLUSTER, int TOK>
 __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorMap* tmap_y, uint32_t tmem_base,
                                               uint8_t* stage, float* sx_slice, int warp, int lane, int tile0,
                                               int tile_step, int num_tiles, int ch_per_tile, int ch_offset,
                                               uint32_t acc_full, uint32_t acc_empty, uint64_t limit,
                                               volatile int* abort_flag) {
   using O = OutTraits<OUT>;
+  constexpr int kEpiCols = TOK / 2;   // tokens of one epilogue warp per tile
+  static_assert(TOK % 64 == 0 && TOK <= kAccCols, "tile width");
   const int q = warp & 3;         // TMEM lanes 32 q .. 32 q + 31
-  const int h = warp >> 2;        // accumulator columns 128 h .. 128 h + 127
+  const int h = warp >> 2;        // accumulator columns kEpiCols h .. kEpiCols (h + 1) - 1
   const uint32_t stage_addr = ptx::smem_addr(stage);
   uint32_t as = 0, aph = 0;
   bool store_pending = false;
@@ -97,7 +99,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
   for (int tile = tile0; tile < num_tiles; tile += tile_step) {
     const int mt = tile % g.num_m_tiles;
     const int nt = tile / g.num_m_tiles;
-    const int tok0 = mt * kAccCols + h * kEpiCols;
+    const int tok0 = mt * TOK + h * kEpiCols;
     const bool got = ptx::wait_bounded(acc_full + 8u * as, aph, limit, abort_flag);
     if (!__all_sync(0xffffffffu, got)) {
       if (lane == 0) raise_failure(g.status, abort_flag, TASQ_DEVICE_TIMEOUT_EPILOGUE);
@@ -105,7 +107,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
     }
     ptx::tc_fence_after_sync();
     const int c0 = nt * ch_per_tile + ch_offset + q * 32;   // first channel of this warp
-    const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + as * kAccCols + h * kEpiCols;
+    const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + as * TOK + h * kEpiCols;
     if constexpr (O::kS32) {
       const int ch = c0 + lane;
 #pragma unroll 1
@@ -159,8 +161,8 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
           sw[gg][o] = ch < g.N ? g.s_w[ch] : 0.0f;
         }
       }
-      // this warp's 128 token scales, read once per tile into its private slice
-      {
+      // this warp's token scales, read once per tile into its private slice
+      if (4 * lane < kEpiCols) {
         float4 v4;
         const int m = tok0 + 4 * lane;
         v4.x = m < g.M ? g.s_x[m] : 0.0f;
@@ -168,8 +170,8 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
         v4.z = m + 2 < g.M ? g.s_x[m + 2] : 0.0f;
         v4.w = m + 3 < g.M ? g.s_x[m + 3] : 0.0f;
         reinterpret_cast<float4*>(sx_slice)[lane] = v4;
-        __syncwarp();
       }
+      __syncwarp();
 #pragma unroll 1
       for (int j = 0; j < kEpiCols / 32; ++j) {
         uint32_t ra[16], rb[16];   // lanes 32 q + 0 .. 15 and 32 q + 16 .. 31

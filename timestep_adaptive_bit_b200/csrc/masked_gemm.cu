@@ -17,9 +17,11 @@
 //                   stages of 128 bytes = four tcgen05.mma.kind::i8 of K = 32.
 //   warp 8          TMA producer: loads the 16 KB weight tile and the 32 KB code tile of each
 //                   stage into 128-byte-swizzled shared memory (4 stages in flight).
-//   warps 10-13     mask warps (only when k > 0): AND every weight byte of a landed stage with
-//                   0xFF << k in place (layout-agnostic, 8 x 16 B per thread), fence the
-//                   generic-proxy writes to the async proxy and release the stage to the MMA.
+//   warps 10-17     mask warps, two groups of four taking alternate K blocks (only when k > 0
+//                   and the weights were not masked ahead by the prologue launch): AND every
+//                   weight byte of a landed stage with 0xFF << k in place (layout-agnostic,
+//                   8 x 16 B per thread), fence the generic-proxy writes to the async proxy and
+//                   release the stage to the MMA.
 //   warp 9          TMEM allocation (512 columns = two 256-column INT32 accumulators) and the
 //                   single MMA-issuing thread; tcgen05.commit frees stages and publishes
 //                   finished accumulators.
@@ -40,16 +42,18 @@ namespace {
 using namespace gemm;
 
 constexpr int kTileCh = kGemmTileCh;      // 128 output channels per tile
-constexpr int kTileTok = kGemmTileTok;    // 256 tokens per tile
 constexpr int kABytes = kTileCh * kBlockK;
-constexpr int kBBytes = kTileTok * kBlockK;
-constexpr int kStageBytes = kABytes + kBBytes;
-static_assert(kTileTok == kAccCols, "accumulator width");
+constexpr int kMaskGroups = 2;            // groups of kMaskWarps mask warps, alternate K blocks
+constexpr int kThreads1 = kThreads + 32 * kMaskWarps * (kMaskGroups - 1);
+static_assert(kABytes % (16 * kMaskThreads) == 0, "mask pass must tile the weight stage");
 
 // Shared-memory plan of one instantiation: stages of (weights, codes), the epilogue's output
 // staging (one 32 x 32 box per warp), its s_x slices, the barriers.
 template <int OUT>
 struct Plan {
+  static constexpr int kTok = kGemmTileTok;
+  static constexpr int kBBytes = kTok * kBlockK;
+  static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = OutTraits<OUT>::kS32 ? 3 : 4;
   static constexpr int kEpiOffset = kStages * kStageBytes;
   static constexpr int kSxOffset = kEpiOffset + kEpiWarps * OutTraits<OUT>::kStageBytes;
@@ -57,9 +61,9 @@ struct Plan {
   static constexpr int kNumBars = 3 * kStages + 2 * kAccStages + 1;
   static constexpr int kSmemBytes = 1024 /* alignment slack */ + kBarOffset + kNumBars * 8 + 16;
   static_assert(kSmemBytes <= kMaxSmem, "shared memory");
+  static_assert(kAccStages * kTok <= static_cast<int>(kTmemCols), "TMEM");
+  static_assert(kStages >= kMaskGroups, "one stage per mask group");
 };
-
-static_assert(kABytes % (16 * kMaskThreads) == 0, "mask pass must tile the weight stage");
 
 template <int STAGES>
 struct Bars {
@@ -73,11 +77,12 @@ struct Bars {
 };
 
 template <int OUT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads1, 1)
     masked_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                        const __grid_constant__ CUtensorMap tmap_y, const GemmArgs g) {
   using P = Plan<OUT>;
   constexpr int kStages = P::kStages;
+  constexpr int kTok = P::kTok;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = ptx::smem_addr(smem);
@@ -97,7 +102,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bits = 8;
   }
   const int k_drop = 8 - bits;
-  const bool masking = k_drop > 0;
+  // weights masked ahead of this kernel need no pass here
+  const bool masking = k_drop > 0 && g.premasked == 0;
   const uint32_t mask32 = 0x01010101u * ((0xFFu << k_drop) & 0xFFu);
 
   if (threadIdx.x == 0) {
@@ -149,9 +155,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          ptx::mbar_arrive_expect_tx(bars.full(s), kStageBytes);
+          ptx::mbar_arrive_expect_tx(bars.full(s), P::kStageBytes);
           ptx::tma_load_2d(a_base + s * kABytes, &tmap_w, bars.full(s), kb * kBlockK, nt * kTileCh);
-          ptx::tma_load_2d(b_base + s * kBBytes, &tmap_x, bars.full(s), kb * kBlockK, mt * kTileTok);
+          ptx::tma_load_2d(b_base + s * P::kBBytes, &tmap_x, bars.full(s), kb * kBlockK, mt * kTok);
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
           if (++s == kStages) {
@@ -171,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       // ------------------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = ptx::idesc_i8_s32(kTileCh, kTileTok);
+      constexpr uint32_t idesc = ptx::idesc_i8_s32(kTileCh, kTok);
       uint32_t s = 0, ph = 0, as = 0, aph = 0;
       bool ok = true;
       bool issued_any = false;
@@ -181,17 +187,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         ptx::tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_base + as * kAccCols;
+        const uint32_t d_tmem = tmem_base + as * kTok;
         for (int kb = 0; kb < g.num_kb; ++kb) {
-          const uint32_t ready = masking ? bars.masked(s) : bars.full(s);
-          if (!ptx::wait_bounded(ready, ph, limit, abort_flag)) {
+          if (!ptx::wait_bounded(masking ? bars.masked(s) : bars.full(s), ph, limit, abort_flag)) {
             raise_failure(g.status, abort_flag, TASQ_DEVICE_TIMEOUT_MMA);
             ok = false;
             break;
           }
           ptx::tc_fence_after_sync();
           const uint64_t a_desc = ptx::smem_desc_k_sw128(a_base + s * kABytes);
-          const uint64_t b_desc = ptx::smem_desc_k_sw128(b_base + s * kBBytes);
+          const uint64_t b_desc = ptx::smem_desc_k_sw128(b_base + s * P::kBBytes);
 #pragma unroll
           for (int kk = 0; kk < kBlockK / kUmmaK; ++kk) {
             // +32 bytes along K inside the 128-byte swizzle row = +2 in the address field
@@ -218,12 +223,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kMaskWarp0) {
     // -------------------------------------------------------------------- mask warps
+    // Two groups of four warps take alternate K blocks of the CTA's sequence (group 0 the even
+    // ones), so that one group's load-mask-store latency overlaps the other's.
+    const int grp = (warp - kMaskWarp0) / kMaskWarps;
+    const int t = threadIdx.x - (kMaskWarp0 + grp * kMaskWarps) * 32;
+    // stage s of this group's next K block, and its phase
+    uint32_t s = grp, ph = 0;
+    uint32_t seq = 0;   // K blocks of the CTA's sequence so far
+    bool ok = true;
     if (masking) {
-      const int t = threadIdx.x - kMaskWarp0 * 32;
-      uint32_t s = 0, ph = 0;
-      bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        for (int kb = 0; kb < g.num_kb; ++kb) {
+        for (int kb = 0; kb < g.num_kb; ++kb, ++seq) {
+          if (static_cast<int>(seq % kMaskGroups) != grp) continue;
           if (!ptx::wait_bounded(bars.full(s), ph, limit, abort_flag)) {
             raise_failure(g.status, abort_flag, TASQ_DEVICE_TIMEOUT_MASK);
             ok = false;
@@ -233,8 +244,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(bars.masked(s));
-          if (++s == kStages) {
-            s = 0;
+          s += kMaskGroups;
+          if (s >= static_cast<uint32_t>(kStages)) {
+            s -= kStages;
             ph ^= 1u;
           }
         }
@@ -242,10 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------------------------- epilogue warps
-    epilogue_role<OUT, false>(g, &tmap_y, tmem_base, smem + P::kEpiOffset + warp * OutTraits<OUT>::kStageBytes,
-                              reinterpret_cast<float*>(smem + P::kSxOffset + warp * kSxBytesPerWarp), warp, lane,
-                              blockIdx.x, gridDim.x, num_tiles, kTileCh, 0, bars.acc_full(0), bars.acc_empty(0),
-                              limit, abort_flag);
+    epilogue_role<OUT, false, kTok>(g, &tmap_y, tmem_base, smem + P::kEpiOffset + warp * OutTraits<OUT>::kStageBytes,
+                                    reinterpret_cast<float*>(smem + P::kSxOffset + warp * kSxBytesPerWarp), warp,
+                                    lane, blockIdx.x, gridDim.x, num_tiles, kTileCh, 0, bars.acc_full(0),
+                                    bars.acc_empty(0), limit, abort_flag);
   }
 
   __syncwarp();
@@ -275,7 +287,7 @@ cudaError_t launch_out(const CUtensorMap& tw, const CUtensorMap& tx, const CUten
   const int grid = tiles < num_sms ? tiles : num_sms;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(kThreads1, 1, 1);
   cfg.dynamicSmemBytes = Plan<OUT>::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

@@ -9,10 +9,11 @@
 // channels x 256 tokens. Per SM and per K stage this moves half the activation bytes of the
 // one-CTA tile through shared memory and L2 for the same number of MACs.
 //
-// Roles per CTA (448 threads), as in the one-CTA kernel:
+// Roles per CTA (448 threads), as in the one-CTA kernel but with one group of mask warps:
 //   warp 8      TMA producer of this CTA's halves, completion on its own `full` barrier.
-//   warps 10-13 apply the step's LSB mask to this CTA's weight half in place (when k > 0) and
-//               then arrive on the first CTA's `ready` barrier (one arrival per warp).
+//   warps 10-13 apply the step's LSB mask to this CTA's weight half in place (when k > 0 and the
+//               weights were not masked ahead by the prologue launch) and then arrive on the
+//               first CTA's `ready` barrier (one arrival per warp).
 //   warp 9      TMEM allocation for the pair (both CTAs); in the first CTA also the MMA thread,
 //               which commits stage and accumulator completion to the barriers of both CTAs.
 //   warps 0-7   epilogue of this CTA's 128 channels; each warp arrives once on the first CTA's
@@ -90,7 +91,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bits = 8;
   }
   const int k_drop = 8 - bits;
-  const bool masking = k_drop > 0;
+  // weights masked ahead of this kernel need no pass here
+  const bool masking = k_drop > 0 && g.premasked == 0;
   const uint32_t mask32 = 0x01010101u * ((0xFFu << k_drop) & 0xFFu);
 
   if (threadIdx.x == 0) {
@@ -245,7 +247,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------------------------- epilogue warps
-    epilogue_role<OUT, true>(g, &tmap_y, tmem_base, smem + P::kEpiOffset + warp * OutTraits<OUT>::kStageBytes,
+    epilogue_role<OUT, true, kPairTok>(g, &tmap_y, tmem_base, smem + P::kEpiOffset + warp * OutTraits<OUT>::kStageBytes,
                              reinterpret_cast<float*>(smem + P::kSxOffset + warp * kSxBytesPerWarp), warp, lane,
                              pair_id, num_pairs, num_tiles, kPairCh, static_cast<int>(rank) * kHalf,
                              bars.acc_full(0), ptx::mapa_shared(bars.acc_empty(0), 0), limit, abort_flag);

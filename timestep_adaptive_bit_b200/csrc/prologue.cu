@@ -21,6 +21,12 @@
 // are the same bits as a textbook FP32 fast Walsh-Hadamard transform produces.
 // The per-row absmax is combined through a shared-memory atomicMax on the float bits (all values
 // are non-negative). No FMA contraction happens anywhere on the path.
+//
+// The same launch can also truncate a layer's weights for the step (TASQ's LSB mask,
+// w AND (0xFF << k) with k = 8 - bits): CTAs past the activation rows stream the layer's INT8
+// weights once, 32 bytes per thread and load, into a masked copy that the GEMM then reads as its
+// weight operand. Masking once per forward costs 2 N Kp bytes of HBM traffic; masking inside the
+// GEMM costs a shared-memory read and write of every weight tile for every token tile.
 #include <cuda_fp16.h>
 
 #include "tasq_internal.h"
@@ -107,9 +113,50 @@ __device__ __forceinline__ float2 fma2_sign(float2 mine, float s, float2 other) 
   return *reinterpret_cast<const float2*>(&r);
 }
 
+constexpr int kWeightUnroll = 4;         // 32-byte loads in flight per thread in the weight pass
+constexpr int64_t kMaxWeightCtas = 592;  // four CTAs for each of a B200's 148 SMs
+
+// Weight pass of CTA `cta` of `num_ctas`: w_dst = w_src AND the step's byte mask.
+__device__ __forceinline__ void weight_pass(const PrologueArgs& a, int64_t cta, int64_t num_ctas) {
+  // the previous GEMM may still read w_dst: wait for it, then let the next kernel start its setup
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  int bits = a.bits_table[a.bits_index];
+  if (bits < 1 || bits > 8) {
+    if (cta == 0 && threadIdx.x == 0) atomicOr(a.status, TASQ_DEVICE_BAD_BITS);
+    bits = 8;
+  }
+  const uint32_t m = 0x01010101u * ((0xFFu << (8 - bits)) & 0xFFu);
+  const int64_t n32 = a.w_bytes >> 5;
+  const int64_t stride = num_ctas * blockDim.x;
+  for (int64_t i0 = cta * blockDim.x + threadIdx.x; i0 < n32; i0 += kWeightUnroll * stride) {
+    uint32_t u[kWeightUnroll][8];
+#pragma unroll
+    for (int j = 0; j < kWeightUnroll; ++j) {
+      const int64_t i = i0 + j * stride;
+      if (i < n32) ld_32B(a.w_src + 32 * i, u[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < kWeightUnroll; ++j) {
+      const int64_t i = i0 + j * stride;
+      if (i < n32) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) u[j][e] &= m;
+        st_32B(a.w_dst + 32 * i, u[j]);
+      }
+    }
+  }
+}
+
 // LANES = n / 32 lanes per Hadamard block; VEC32: row starts of x and xq are 32-byte aligned.
+// CTAs [0, row_ctas) quantize activation rows, the rest run the weight pass.
 template <int LANES, bool VEC32>
-__global__ void __launch_bounds__(kMaxThreads) prologue_kernel(const PrologueArgs a, const int rows_per_cta) {
+__global__ void __launch_bounds__(kMaxThreads)
+    prologue_kernel(const PrologueArgs a, const int rows_per_cta, const int row_ctas) {
+  if (static_cast<int>(blockIdx.x) >= row_ctas) {
+    weight_pass(a, blockIdx.x - row_ctas, gridDim.x - row_ctas);
+    return;
+  }
   const int L = a.Kp >> 5;                       // 32-channel segments per row
   const int tid = threadIdx.x;
   const int r_local = tid / L;
@@ -242,15 +289,31 @@ int pick_rows(int C) {
 }  // namespace
 
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
-  if (a.M <= 0) return cudaSuccess;
+  const bool weights = a.w_bytes > 0;
+  if (a.M <= 0 && !weights) return cudaSuccess;
   if (a.Kp % a.n != 0 || (a.n != 64 && a.n != 128)) return cudaErrorInvalidValue;
+  if (weights && (a.w_bytes % 32 != 0 || reinterpret_cast<uintptr_t>(a.w_src) % 32 != 0 ||
+                  reinterpret_cast<uintptr_t>(a.w_dst) % 32 != 0 || a.bits_table == nullptr || a.status == nullptr))
+    return cudaErrorInvalidValue;
   const int L = a.Kp / 32;
   if (L > kMaxThreads) return cudaErrorInvalidValue;
-  const int R = pick_rows(L);
-  const int threads = ((R * L + 31) / 32) * 32;
-  const int64_t grid = (a.M + R - 1) / R;
+  int R = 1, threads = 256;
+  int64_t row_ctas = 0;
+  if (a.M > 0) {
+    R = pick_rows(L);
+    threads = ((R * L + 31) / 32) * 32;
+    row_ctas = (a.M + R - 1) / R;
+  }
+  int64_t weight_ctas = 0;
+  if (weights) {
+    // about kWeightUnroll 32-byte loads per thread; larger layers loop
+    const int64_t per_cta = static_cast<int64_t>(threads) * 32 * kWeightUnroll;
+    weight_ctas = (a.w_bytes + per_cta - 1) / per_cta;
+    if (weight_ctas > kMaxWeightCtas) weight_ctas = kMaxWeightCtas;
+  }
+  const int64_t grid = row_ctas + weight_ctas;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
-  const bool vec32 = (reinterpret_cast<uintptr_t>(a.x) % 32 == 0) && (a.ldx % 16 == 0) &&
+  const bool vec32 = a.M > 0 && (reinterpret_cast<uintptr_t>(a.x) % 32 == 0) && (a.ldx % 16 == 0) &&
                      (reinterpret_cast<uintptr_t>(a.xq) % 32 == 0);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
@@ -261,12 +324,13 @@ cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = use_pdl() ? 1 : 0;
+  const int rc = static_cast<int>(row_ctas);
   if (a.n == 64) {
-    if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<2, true>, a, R);
-    return cudaLaunchKernelEx(&cfg, prologue_kernel<2, false>, a, R);
+    if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<2, true>, a, R, rc);
+    return cudaLaunchKernelEx(&cfg, prologue_kernel<2, false>, a, R, rc);
   }
-  if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<4, true>, a, R);
-  return cudaLaunchKernelEx(&cfg, prologue_kernel<4, false>, a, R);
+  if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<4, true>, a, R, rc);
+  return cudaLaunchKernelEx(&cfg, prologue_kernel<4, false>, a, R, rc);
 }
 
 }  // namespace tasq

@@ -137,6 +137,13 @@ struct tasq_ctx {
   uint64_t wait_limit_ns = 1000000000ull;
   float sx_factor = 0.0f;
   int32_t gemm_mode = 0;   // 0 automatic, 1 one CTA per tile, 2 CTA pairs
+  int32_t mask_mode = 0;   // 0 automatic, 1 mask inside the GEMM, 2 mask ahead in the prologue launch
+  // host copy of the last schedule given, used only to choose where the mask is applied: both
+  // places read the device table and give the same result for every bit width, so a device table
+  // that is newer or older than this copy changes no result
+  std::vector<uint8_t> bits_host;
+  int8_t* d_wk = nullptr;              // masked copy of one layer's weights (largest N x Kp)
+  std::vector<CUtensorMap> tmap_wk;    // per layer, over d_wk
   // trace
   int32_t trace_cap = 0, trace_count = 0;
   std::vector<TraceRec> trace;
@@ -149,6 +156,7 @@ void free_ctx(tasq_ctx* c) {
   if (c->device >= 0) cudaSetDevice(c->device);
   cudaDeviceSynchronize();
   cudaFree(c->d_w);
+  cudaFree(c->d_wk);
   cudaFree(c->d_sw);
   cudaFree(c->d_bits);
   cudaFree(c->d_xq);
@@ -203,9 +211,32 @@ tasq_status check_rows(const void* p, int64_t ld, int64_t width, const char* nam
   return TASQ_OK;
 }
 
-tasq_status run_prologue(tasq_ctx* c, const LayerInfo& L, const void* x, int64_t M, int64_t ldx, int8_t* xq, float* sx,
-                         cudaStream_t s) {
+// Whether this forward masks the layer's weights once in the prologue launch (true) or lets the
+// GEMM mask every weight tile it loads (false). Masking ahead pays whenever the step drops bits;
+// at 8 bits the GEMM reads the stored weights directly.
+bool mask_ahead(const tasq_ctx* c, int32_t layer, int32_t step) {
+  if (c->mask_mode != 0) return c->mask_mode == 2;
+  return c->bits_host[static_cast<size_t>(layer) * c->num_steps + step] < 8;
+}
+
+// The prologue launch's weight-pass fields for (layer, step).
+void set_weight_pass(tasq::PrologueArgs& a, const tasq_ctx* c, int32_t layer, int32_t step) {
+  const LayerInfo& L = c->layers[layer];
+  a.w_src = c->d_w + L.w_off;
+  a.w_dst = c->d_wk;
+  a.w_bytes = static_cast<int64_t>(L.N) * L.Kp;
+  a.bits_table = c->d_bits;
+  a.bits_index = layer * c->num_steps + step;
+  a.status = c->d_status;
+}
+
+// Activation prologue of (layer, step) over M rows (M may be 0), with the weight pass when
+// `weights` is set.
+tasq_status run_prologue(tasq_ctx* c, int32_t layer, int32_t step, bool weights, const void* x, int64_t M,
+                         int64_t ldx, int8_t* xq, float* sx, cudaStream_t s) {
+  const LayerInfo& L = c->layers[layer];
   tasq::PrologueArgs a{};
+  if (weights) set_weight_pass(a, c, layer, step);
   a.x = x;
   a.ldx = ldx;
   a.K = L.K;
@@ -235,12 +266,14 @@ bool prefer_pair(int64_t M, int64_t N, int num_sms) {
 }
 
 tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq, const float* sx, int64_t M,
-                     void* y, int64_t ldy, tasq::OutKind out, cudaStream_t s) {
+                     void* y, int64_t ldy, tasq::OutKind out, bool premasked, cudaStream_t s) {
   const LayerInfo& L = c->layers[layer];
   const bool pair = c->gemm_mode == 2 || (c->gemm_mode == 0 && prefer_pair(M, L.N, c->num_sms));
+  const int tile_tok = pair ? tasq::kGemmPairTile : tasq::kGemmTileTok;
+  const int tile_ch = pair ? tasq::kGemmPairTile : tasq::kGemmTileCh;
   CUtensorMap tx;
   tasq_status st = make_tmap_u8(&tx, xq, static_cast<uint64_t>(L.Kp), static_cast<uint64_t>(M), tasq::kGemmBlockK,
-                                pair ? tasq::kGemmPairHalf : tasq::kGemmTileTok);
+                                pair ? tasq::kGemmPairHalf : tile_tok);
   if (st != TASQ_OK) return st;
   CUtensorMap ty;
   const CUtensorMapDataType dt = out == tasq::OutKind::S32    ? CU_TENSOR_MAP_DATA_TYPE_INT32
@@ -253,8 +286,6 @@ tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq,
   g.M = static_cast<int32_t>(M);
   g.N = L.N;
   g.num_kb = (L.Kp + tasq::kGemmBlockK - 1) / tasq::kGemmBlockK;
-  const int tile_tok = pair ? tasq::kGemmPairTile : tasq::kGemmTileTok;
-  const int tile_ch = pair ? tasq::kGemmPairTile : tasq::kGemmTileCh;
   g.num_m_tiles = static_cast<int32_t>((M + tile_tok - 1) / tile_tok);
   g.num_n_tiles = (L.N + tile_ch - 1) / tile_ch;
   g.bits_table = c->d_bits;
@@ -265,10 +296,21 @@ tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq,
   g.ldy = ldy;
   g.status = c->d_status;
   g.wait_limit_ns = c->wait_limit_ns;
-  cudaError_t e = pair ? tasq::launch_masked_gemm_pair(c->tmap_w[layer], tx, ty, g, out, c->num_sms, s)
-                       : tasq::launch_masked_gemm(c->tmap_w[layer], tx, ty, g, out, c->num_sms, s);
+  g.premasked = premasked ? 1 : 0;
+  const CUtensorMap& tw = premasked ? c->tmap_wk[layer] : c->tmap_w[layer];
+  cudaError_t e = pair ? tasq::launch_masked_gemm_pair(tw, tx, ty, g, out, c->num_sms, s)
+                       : tasq::launch_masked_gemm(tw, tx, ty, g, out, c->num_sms, s);
   if (e != cudaSuccess) return fail_cuda(e, "masked GEMM launch");
   return TASQ_OK;
+}
+
+// GEMM of given codes, with the weight pass launched alone first when the mask goes ahead.
+tasq_status debug_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq, const float* sx, int64_t M, void* y,
+                       int64_t ldy, tasq::OutKind out, cudaStream_t s) {
+  const bool ahead = mask_ahead(c, layer, step);
+  tasq_status st;
+  if (ahead && (st = run_prologue(c, layer, step, true, nullptr, 0, 0, nullptr, nullptr, s)) != TASQ_OK) return st;
+  return run_gemm(c, layer, step, xq, sx, M, y, ldy, out, ahead, s);
 }
 
 }  // namespace
@@ -303,7 +345,7 @@ tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, in
                                                std::to_string(prop.minor) + ", this library is built for sm_100a");
 
   std::vector<LayerInfo> info(num_layers);
-  size_t w_bytes = 0, sw_count = 0;
+  size_t w_bytes = 0, sw_count = 0, wk_bytes = 0;
   int32_t kp_max = 0;
   for (int32_t l = 0; l < num_layers; ++l) {
     const tasq_layer_desc& d = layers[l];
@@ -317,6 +359,7 @@ tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, in
                                             " exceeds " + std::to_string(TASQ_MAX_KP));
     info[l] = LayerInfo{d.N, d.K, Kp, w_bytes, sw_count};
     w_bytes = round_up(w_bytes + static_cast<size_t>(d.N) * Kp, 1024);
+    if (static_cast<size_t>(d.N) * Kp > wk_bytes) wk_bytes = static_cast<size_t>(d.N) * Kp;
     sw_count = round_up(sw_count + d.N, 64);
     if (Kp > kp_max) kp_max = Kp;
   }
@@ -340,6 +383,7 @@ tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, in
     return st;
   };
   if ((e = cudaMalloc(&c->d_w, w_bytes)) != cudaSuccess) return bail(e, "cudaMalloc(weights)");
+  if ((e = cudaMalloc(&c->d_wk, wk_bytes)) != cudaSuccess) return bail(e, "cudaMalloc(masked weights)");
   if ((e = cudaMalloc(&c->d_sw, sw_count * sizeof(float))) != cudaSuccess) return bail(e, "cudaMalloc(scales)");
   const size_t table = static_cast<size_t>(num_layers) * num_steps;
   if ((e = cudaMalloc(&c->d_bits, table)) != cudaSuccess) return bail(e, "cudaMalloc(schedule)");
@@ -350,6 +394,7 @@ tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, in
   if ((e = cudaMalloc(&c->d_status, sizeof(uint32_t))) != cudaSuccess) return bail(e, "cudaMalloc(status)");
 
   if ((e = cudaMemsetAsync(c->d_bits, 8, table, s)) != cudaSuccess) return bail(e, "cudaMemsetAsync(schedule)");
+  c->bits_host.assign(table, 8);
   if ((e = cudaMemsetAsync(c->d_status, 0, sizeof(uint32_t), s)) != cudaSuccess) return bail(e, "cudaMemsetAsync(status)");
   for (int32_t l = 0; l < num_layers; ++l) {
     const LayerInfo& L = info[l];
@@ -362,10 +407,14 @@ tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, in
   if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return bail(e, "cudaStreamSynchronize");
 
   c->tmap_w.resize(num_layers);
+  c->tmap_wk.resize(num_layers);
   for (int32_t l = 0; l < num_layers; ++l) {
     const LayerInfo& L = info[l];
     tasq_status st = make_tmap_u8(&c->tmap_w[l], c->d_w + L.w_off, static_cast<uint64_t>(L.Kp),
                                   static_cast<uint64_t>(L.N), tasq::kGemmBlockK, tasq::kGemmTileCh);
+    if (st == TASQ_OK)
+      st = make_tmap_u8(&c->tmap_wk[l], c->d_wk, static_cast<uint64_t>(L.Kp), static_cast<uint64_t>(L.N),
+                        tasq::kGemmBlockK, tasq::kGemmTileCh);
     if (st != TASQ_OK) {
       std::string m = g_last_error;
       free_ctx(c);
@@ -389,6 +438,7 @@ tasq_status tasq_set_schedule(tasq_ctx* c, const uint8_t* bits_host, void* strea
   }
   cudaError_t e = cudaMemcpyAsync(c->d_bits, bits_host, table, cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e, "copy of schedule");
+  c->bits_host.assign(bits_host, bits_host + table);
   return TASQ_OK;
 }
 
@@ -408,15 +458,16 @@ tasq_status tasq_linear_forward(tasq_ctx* c, const void* x, int64_t M, int64_t l
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   TraceRec* tr = c->trace_count < c->trace_cap ? &c->trace[c->trace_count] : nullptr;
+  const bool ahead = mask_ahead(c, layer, step);
   if (tr) cudaEventRecord(tr->e0, s);
-  if ((st = run_prologue(c, L, x, M, ldx, c->d_xq, c->d_sx, s)) != TASQ_OK) return st;
+  if ((st = run_prologue(c, layer, step, ahead, x, M, ldx, c->d_xq, c->d_sx, s)) != TASQ_OK) return st;
   if (tr) cudaEventRecord(tr->e1, s);
   const tasq::OutKind out = c->out_dtype == TASQ_OUT_BF16 ? tasq::OutKind::BF16 : tasq::OutKind::F16;
-  if ((st = run_gemm(c, layer, step, c->d_xq, c->d_sx, M, y, ldy, out, s)) != TASQ_OK) return st;
+  if ((st = run_gemm(c, layer, step, c->d_xq, c->d_sx, M, y, ldy, out, ahead, s)) != TASQ_OK) return st;
   if (tr) {
     cudaEventRecord(tr->e2, s);
     tr->ops = 2.0 * static_cast<double>(M) * L.N * L.K;
-    tr->bytes = static_cast<double>(M) * (2.0 * L.K + L.Kp + 4.0);
+    tr->bytes = static_cast<double>(M) * (2.0 * L.K + L.Kp + 4.0) + (ahead ? 2.0 * L.N * L.Kp : 0.0);
     ++c->trace_count;
   }
   return TASQ_OK;
@@ -480,7 +531,7 @@ tasq_status tasq_debug_quantize(tasq_ctx* c, const void* x, int64_t M, int64_t l
   if (s_x == nullptr || !aligned16(s_x)) return fail(TASQ_ERR_INVALID_ARG, "s_x must be a 16-byte aligned pointer");
   if ((st = check_device(c)) != TASQ_OK) return st;
   if (M == 0) return TASQ_OK;
-  return run_prologue(c, L, x, M, ldx, xq, s_x, static_cast<cudaStream_t>(stream));
+  return run_prologue(c, layer, 0, false, x, M, ldx, xq, s_x, static_cast<cudaStream_t>(stream));
 }
 
 tasq_status tasq_debug_gemm_s32(tasq_ctx* c, const int8_t* xq, int64_t M, int32_t layer, int32_t step, int32_t* acc,
@@ -496,7 +547,7 @@ tasq_status tasq_debug_gemm_s32(tasq_ctx* c, const int8_t* xq, int64_t M, int32_
   if ((st = check_rows(acc, ld_acc, L.N, "acc")) != TASQ_OK) return st;
   if ((st = check_device(c)) != TASQ_OK) return st;
   if (M == 0) return TASQ_OK;
-  return run_gemm(c, layer, step, xq, nullptr, M, acc, ld_acc, tasq::OutKind::S32, static_cast<cudaStream_t>(stream));
+  return debug_gemm(c, layer, step, xq, nullptr, M, acc, ld_acc, tasq::OutKind::S32, static_cast<cudaStream_t>(stream));
 }
 
 tasq_status tasq_debug_gemm(tasq_ctx* c, const int8_t* xq, const float* s_x, int64_t M, int32_t layer, int32_t step,
@@ -515,7 +566,7 @@ tasq_status tasq_debug_gemm(tasq_ctx* c, const int8_t* xq, const float* s_x, int
   if ((st = check_device(c)) != TASQ_OK) return st;
   if (M == 0) return TASQ_OK;
   const tasq::OutKind out = out_dtype == TASQ_OUT_BF16 ? tasq::OutKind::BF16 : tasq::OutKind::F16;
-  return run_gemm(c, layer, step, xq, s_x, M, y, ldy, out, static_cast<cudaStream_t>(stream));
+  return debug_gemm(c, layer, step, xq, s_x, M, y, ldy, out, static_cast<cudaStream_t>(stream));
 }
 
 tasq_status tasq_debug_set_gemm_mode(tasq_ctx* c, int32_t mode) {
@@ -523,6 +574,14 @@ tasq_status tasq_debug_set_gemm_mode(tasq_ctx* c, int32_t mode) {
   if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
   if (mode < 0 || mode > 2) return fail(TASQ_ERR_INVALID_ARG, "mode must be 0, 1 or 2");
   c->gemm_mode = mode;
+  return TASQ_OK;
+}
+
+tasq_status tasq_debug_set_mask_mode(tasq_ctx* c, int32_t mode) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  if (mode < 0 || mode > 2) return fail(TASQ_ERR_INVALID_ARG, "mode must be 0, 1 or 2");
+  c->mask_mode = mode;
   return TASQ_OK;
 }
 

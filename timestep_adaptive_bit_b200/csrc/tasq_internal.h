@@ -22,7 +22,19 @@ struct PrologueArgs {
   float* s_x;         // [M]
   int32_t n;          // 64 or 128
   float sx_factor;    // fp32(1 / (127 sqrt(n)))
+  // Optional weight pass in the same launch (w_bytes > 0): w_dst = w_src AND the byte mask
+  // 0xFF << (8 - bits), bits = bits_table[bits_index]; out-of-range bits set
+  // TASQ_DEVICE_BAD_BITS in *status and are read as 8. Both buffers 32-byte aligned, w_bytes a
+  // multiple of 32.
+  const int8_t* w_src;
+  int8_t* w_dst;
+  int64_t w_bytes;
+  const uint8_t* bits_table;
+  int32_t bits_index;
+  uint32_t* status;
 };
+// Launches the activation rows (M > 0) and the weight pass (w_bytes > 0) as one grid; either
+// part may be empty.
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream);
 
 enum class OutKind : int { F16 = 0, BF16 = 1, S32 = 2 };
@@ -42,6 +54,7 @@ struct GemmArgs {
   int64_t ldy;
   uint32_t* status;
   uint64_t wait_limit_ns;
+  int32_t premasked;       // 1: the weight operand already holds mask(w) for this bit width
 };
 cudaError_t launch_masked_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const CUtensorMap& tmap_y,
                                const GemmArgs& g, OutKind out, int num_sms, cudaStream_t stream);
