@@ -63,6 +63,8 @@ def parse_args(argv=None):
                    help="GEMM kernel: 0 automatic, 1 one CTA per tile, 2 CTA pairs")
     p.add_argument("--mask-mode", type=int, default=0, choices=[0, 1, 2],
                    help="LSB mask: 0 automatic, 1 inside the GEMM on every tile, 2 once ahead in the prologue launch")
+    p.add_argument("--prologue-mode", type=int, default=0, choices=[0, 1, 2],
+                   help="prologue kernel: 0 automatic, 1 direct loads, 2 bulk-fed ring where it fits")
     return p.parse_args(argv)
 
 
@@ -101,6 +103,16 @@ def profiled_traffic(workload: str):
         with open(os.path.join(ROOT, "timestep_adaptive_bit_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return int(m_t.group(1)) if h.hexdigest() == m_h.group(1) else None
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """Largest `value` over the ranks of the process group (the value itself without one)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def load_peaks():
@@ -240,7 +252,7 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------------------ GPU leg
-def setup_workload(T, torch, wl, device, out_dtype, gemm_mode=0, mask_mode=0):
+def setup_workload(T, torch, wl, device, out_dtype, gemm_mode=0, mask_mode=0, prologue_mode=0):
     """Context with every layer of the workload, one activation buffer per (block, layer),
     one output buffer per distinct N. Weights and activations drawn on the device."""
     L = wl.num_layers
@@ -257,6 +269,7 @@ def setup_workload(T, torch, wl, device, out_dtype, gemm_mode=0, mask_mode=0):
     del keep, layers
     T.tasq_debug_set_gemm_mode(ctx, gemm_mode)
     T.tasq_debug_set_mask_mode(ctx, mask_mode)
+    T.tasq_debug_set_prologue_mode(ctx, prologue_mode)
     T.tasq_set_schedule(ctx, workloads.schedule(wl), stream)
     xs = [workloads.activations_torch(wl, l, device) for l in range(L)]
     tdt = torch.float16 if out_dtype == "f16" else torch.bfloat16
@@ -289,6 +302,7 @@ def profile_case(args):
     ctx = T.tasq_linear_create([(N, K, w, s_w)], 1, wl.hadamard_n, wl.tokens, T.TASQ_OUT_F16, s)
     T.tasq_debug_set_gemm_mode(ctx, args.gemm_mode)
     T.tasq_debug_set_mask_mode(ctx, args.mask_mode)
+    T.tasq_debug_set_prologue_mode(ctx, args.prologue_mode)
     bits = 5 if args.bits is None else args.bits
     T.tasq_set_schedule(ctx, np.array([[bits]], np.uint8), s)
     x = workloads.activations_torch(wl, j, dev)
@@ -317,6 +331,7 @@ def sweep_bits(args):
     ctx = T.tasq_linear_create([(N, K, w, s_w)], 8, wl.hadamard_n, M, T.TASQ_OUT_F16, s)
     T.tasq_debug_set_gemm_mode(ctx, args.gemm_mode)
     T.tasq_debug_set_mask_mode(ctx, args.mask_mode)
+    T.tasq_debug_set_prologue_mode(ctx, args.prologue_mode)
     T.tasq_set_schedule(ctx, np.array([[8, 7, 6, 5, 4, 3, 2, 1]], np.uint8), s)
     # several input buffers so consecutive launches do not find their activations in L2
     nbuf = max(2, int(math.ceil(3 * 126e6 / (M * K * 2))))
@@ -324,7 +339,8 @@ def sweep_bits(args):
     y = torch.empty((M, N), dtype=torch.float16, device=dev)
     peaks, peak_kind = load_peaks()
     out = {"sweep": f"{name}:{wl.block_layers[j][0]}", "M": M, "K": K, "N": N, "reps": args.reps,
-           "gemm_mode": args.gemm_mode, "mask_mode": args.mask_mode, "bits": {}}
+           "gemm_mode": args.gemm_mode, "mask_mode": args.mask_mode, "prologue_mode": args.prologue_mode,
+           "bits": {}}
     for step in range(8):
         for r in range(3):
             T.tasq_linear_forward(ctx, xs[r % nbuf], M, K, 0, step, y, N, s)
@@ -370,14 +386,14 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
 
     wl = workloads.WORKLOADS[args.workload]
-    ctx, xs, ys = setup_workload(T, torch, wl, device, args.out_dtype, args.gemm_mode, args.mask_mode)
+    ctx, xs, ys = setup_workload(T, torch, wl, device, args.out_dtype, args.gemm_mode, args.mask_mode,
+                                 args.prologue_mode)
     stream = torch.cuda.current_stream()
     L = wl.num_layers
 
     for i in range(args.warmup):
         run_step(T, ctx, wl, xs, ys, i % wl.steps, stream)
     torch.cuda.synchronize()
-    T.tasq_trace_enable(ctx, args.steps * L)
     sampler = ClockSampler(local_rank)
     if dist is not None:
         dist.barrier()
@@ -394,13 +410,27 @@ def main(argv=None):
     clocks = sampler.stop()
     if dist is not None:
         dist.barrier()
-    ms = t0.elapsed_time(t1)
-    trace = T.tasq_trace_read(ctx)
-    status = T.tasq_get_device_status(ctx)
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=device)
+    ms_max = max_over_ranks(t0.elapsed_time(t1), dist, device)
+
+    # ---- per-kernel durations: a separate pass of the same steps with CUDA events around every
+    # kernel. Events between the kernels break their programmatic-launch overlap (about 18 % on
+    # the PixArt-Sigma step), so the headline above is timed without them.
+    trace_steps = max(1, min(args.steps, 40))
+    T.tasq_trace_enable(ctx, trace_steps * L)
     if dist is not None:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+        dist.barrier()
+    torch.cuda.synchronize()
+    q0 = torch.cuda.Event(enable_timing=True)
+    q1 = torch.cuda.Event(enable_timing=True)
+    q0.record(stream)
+    for i in range(trace_steps):
+        run_step(T, ctx, wl, xs, ys, i % wl.steps, stream)
+    q1.record(stream)
+    torch.cuda.synchronize()
+    traced_ms = q0.elapsed_time(q1)
+    trace = T.tasq_trace_read(ctx)
+    T.tasq_trace_enable(ctx, 0)
+    status = T.tasq_get_device_status(ctx)
 
     # ---- end to end through the public API: pinned host input in, host result out, per step
     e2e = None
@@ -423,10 +453,7 @@ def main(argv=None):
             y_host.copy_(ys[last_N], non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
-        if dist is not None:
-            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
-        e_ms = float(ems.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
         e2e = {"value": world * e_steps * wl.gemm_ops_per_step() / (e_ms / 1e3) / 1e12, "unit": "TOPS",
                "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
                "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()),
@@ -476,7 +503,10 @@ def main(argv=None):
         "prologue_roofline": {"bound": "hbm", "achieved": pro_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                               "frac": (pro_gbs / peaks["hbm_gbs"]) if pro_gbs else None,
                               "frac_of_8000": (pro_gbs / 8000.0) if pro_gbs else None},
-        "gemm_share_of_step": trace["gemm_ms"] / max(ms, 1e-9) if trace["gemm_ms"] else None,
+        "gemm_share_of_step": trace["gemm_ms"] / max(traced_ms, 1e-9) if trace["gemm_ms"] else None,
+        "kernel_timing": f"per-kernel CUDA events in a separate pass of {trace_steps} steps "
+                         f"({traced_ms / trace_steps:.3f} ms per step with the events); the timed steps run "
+                         "without them",
         "clocks": clocks,
         "gpu_launches": 2 * args.steps * L,
         "device_status": status,

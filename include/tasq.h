@@ -54,6 +54,7 @@ typedef enum {
 #define TASQ_DEVICE_TIMEOUT_MASK 0x4u
 #define TASQ_DEVICE_TIMEOUT_EPILOGUE 0x8u
 #define TASQ_DEVICE_TIMEOUT_DRAIN 0x10u
+#define TASQ_DEVICE_TIMEOUT_PROLOGUE 0x20u
 #define TASQ_DEVICE_BAD_BITS 0x100u
 
 /* Limits of this implementation. */
@@ -185,6 +186,16 @@ tasq_status tasq_debug_set_gemm_mode(tasq_ctx* ctx, int32_t mode);
  * Any other mode is TASQ_ERR_INVALID_ARG.
  */
 tasq_status tasq_debug_set_mask_mode(tasq_ctx* ctx, int32_t mode);
+
+/*
+ * Test hook: which prologue kernel later forwards and tasq_debug_quantize use. 1: the direct-load
+ * kernel (each thread loads its 32 channels straight from global memory, one block of rows per
+ * CTA); 2: the bulk-fed kernel (one persistent CTA per SM, rows streamed into a ring of
+ * shared-memory stages by 1-D bulk copies) wherever its layout fits, else the direct one;
+ * 0 (default): the bulk-fed kernel only when every SM gets many blocks of rows, else the direct
+ * one. All produce bit-identical codes and scales. Any other mode is TASQ_ERR_INVALID_ARG.
+ */
+tasq_status tasq_debug_set_prologue_mode(tasq_ctx* ctx, int32_t mode);
 
 /*
  * Failure-detection hook: launch one CTA that waits, with the context's wait limit, on a

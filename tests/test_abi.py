@@ -48,7 +48,8 @@ def test_enum_and_limits_match_header(tasq):
         m = re.search(rf"\b{name}\s*=\s*(\d+)", src)
         assert m and int(m.group(1)) == getattr(tasq, name), name
     for name in ("TASQ_DEVICE_TIMEOUT_PRODUCER", "TASQ_DEVICE_TIMEOUT_MMA", "TASQ_DEVICE_TIMEOUT_MASK",
-                 "TASQ_DEVICE_TIMEOUT_EPILOGUE", "TASQ_DEVICE_TIMEOUT_DRAIN", "TASQ_DEVICE_BAD_BITS", "TASQ_MAX_KP"):
+                 "TASQ_DEVICE_TIMEOUT_EPILOGUE", "TASQ_DEVICE_TIMEOUT_DRAIN", "TASQ_DEVICE_TIMEOUT_PROLOGUE",
+                 "TASQ_DEVICE_BAD_BITS", "TASQ_MAX_KP"):
         m = re.search(rf"#define\s+{name}\s+(0x[0-9a-fA-F]+|\d+)u?", src)
         assert m and int(m.group(1), 0) == getattr(tasq, name), name
 

@@ -63,9 +63,12 @@ def _ctx(T, layers, steps, n, max_tokens, out=0):
 
 
 # ----------------------------------------------------------------------------- prologue
+# prologue kernels: 1 = direct loads, 2 = bulk-fed ring wherever its layout fits
+@pytest.mark.parametrize("pmode", [1, 2])
 @pytest.mark.parametrize("n,K,M", [(64, 64, 1), (64, 96, 3), (64, 1152, 257), (128, 2240, 130), (128, 128, 5),
-                                   (64, 12288, 33), (128, 16384, 2), (64, 4608, 300), (128, 5600, 64)])
-def test_prologue_matches_oracle(T, n, K, M):
+                                   (64, 12288, 33), (128, 16384, 2), (64, 4608, 300), (128, 5600, 64),
+                                   (64, 1152, 4000), (64, 640, 9001), (128, 3072, 1500)])
+def test_prologue_matches_oracle(T, n, K, M, pmode):
     rng = np.random.default_rng(K * 31 + M)
     x = _acts(rng, M, K)
     if M >= 3:
@@ -73,11 +76,15 @@ def test_prologue_matches_oracle(T, n, K, M):
         x[2] = np.float16(0.5)      # constant token
     Kp = oracle.padded_k(K, n)
     ctx = _ctx(T, [(64, K, np.zeros((64, Kp), np.int8), np.ones(64, np.float32))], 1, n, max(M, 1))
+    T.tasq_debug_set_prologue_mode(ctx, pmode)
     ldx = K + 8                     # strided rows
     xs = np.zeros((M, ldx), np.float16)
     xs[:, :K] = x
     xd = _dev(xs)
-    xq = torch.empty((M, Kp), dtype=torch.int8, device="cuda")
+    # codes 16-byte but not 32-byte aligned for odd M: the narrower store path
+    off = 16 if M % 2 == 1 else 0
+    xq_buf = torch.empty((M * Kp + 64,), dtype=torch.int8, device="cuda")
+    xq = xq_buf[off:off + M * Kp].view(M, Kp)
     sx = torch.empty((M,), dtype=torch.float32, device="cuda")
     T.tasq_debug_quantize(ctx, xd, M, ldx, 0, xq, sx, _stream())
     torch.cuda.synchronize()
@@ -205,6 +212,31 @@ def test_forward_matches_oracle(T, n, K, N, M, mode):
     assert T.tasq_get_device_status(ctx) == 0
 
 
+@pytest.mark.parametrize("n,K,N,M", [(64, 1152, 1152, 300), (128, 5600, 2240, 513), (64, 4608, 640, 2000)])
+def test_forward_bulk_fed_prologue_with_weight_pass(T, n, K, N, M):
+    """The bulk-fed prologue on a whole forward, with the weights masked ahead by the same
+    persistent CTAs after their rows (every step drops bits)."""
+    rng = np.random.default_rng(n + K + N + M + 7)
+    Kp = oracle.padded_k(K, n)
+    x = _acts(rng, M, K)
+    w = rng.integers(-128, 128, size=(N, Kp)).astype(np.int8)
+    s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+    bits_per_step = [7, 4, 1]
+    ctx = _ctx(T, [(N, K, w, s_w)], len(bits_per_step), n, M)
+    T.tasq_debug_set_prologue_mode(ctx, 2)
+    T.tasq_debug_set_mask_mode(ctx, 2)
+    T.tasq_set_schedule(ctx, np.array([bits_per_step], np.uint8), _stream())
+    xd = _dev(x)
+    for step, bits in enumerate(bits_per_step):
+        y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+        T.tasq_linear_forward(ctx, xd, M, K, 0, step, y, N, _stream())
+        torch.cuda.synchronize()
+        got = y.float().cpu().numpy().astype(np.float64)
+        ref = oracle.masked_linear(x, w, s_w, bits, n)["y"]
+        assert np.all(np.abs(got - ref) <= F16_REL * np.abs(ref) + ABS_TINY), f"bits={bits}"
+    assert T.tasq_get_device_status(ctx) == 0
+
+
 def test_schedule_is_stream_ordered(T):
     """A schedule change between two forwards on one stream affects only the later forward, and
     the weights are never rewritten (the same buffer serves both)."""
@@ -312,6 +344,7 @@ def test_argument_errors_on_device(T):
     assert err(T.tasq_debug_set_gemm_mode, ctx, 3) == T.TASQ_ERR_INVALID_ARG
     assert err(T.tasq_debug_set_mask_mode, ctx, 3) == T.TASQ_ERR_INVALID_ARG
     assert err(T.tasq_debug_set_mask_mode, ctx, -1) == T.TASQ_ERR_INVALID_ARG
+    assert err(T.tasq_debug_set_prologue_mode, ctx, 3) == T.TASQ_ERR_INVALID_ARG
     T.tasq_linear_forward(ctx, x, 0, K, 0, 0, y, N, s)        # M = 0: nothing to do
     assert T.tasq_get_device_status(ctx) == 0
     with pytest.raises(T.TasqError):

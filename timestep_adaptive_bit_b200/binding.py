@@ -32,6 +32,7 @@ TASQ_DEVICE_TIMEOUT_MMA = 0x2
 TASQ_DEVICE_TIMEOUT_MASK = 0x4
 TASQ_DEVICE_TIMEOUT_EPILOGUE = 0x8
 TASQ_DEVICE_TIMEOUT_DRAIN = 0x10
+TASQ_DEVICE_TIMEOUT_PROLOGUE = 0x20
 TASQ_DEVICE_BAD_BITS = 0x100
 
 TASQ_MAX_KP = 16384
@@ -71,6 +72,7 @@ def _load():
         "tasq_debug_stuck_wait": [P, P],
         "tasq_debug_set_gemm_mode": [P, i32],
         "tasq_debug_set_mask_mode": [P, i32],
+        "tasq_debug_set_prologue_mode": [P, i32],
         "tasq_trace_enable": [P, i32],
         "tasq_linear_forward_noalloc": [P, i64, i64, i32, P, P, i32, i32, i32, P, i64, i32, P, P],
         "tasq_trace_read": [P, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i32),
@@ -211,6 +213,10 @@ def tasq_debug_gemm(ctx: Context, xq, s_x, M: int, layer: int, step: int, y, ldy
 
 def tasq_debug_set_gemm_mode(ctx: Context, mode: int) -> None:
     _check(lib.tasq_debug_set_gemm_mode(ctx, int(mode)))
+
+
+def tasq_debug_set_prologue_mode(ctx: Context, mode: int) -> None:
+    _check(lib.tasq_debug_set_prologue_mode(ctx, int(mode)))
 
 
 def tasq_debug_set_mask_mode(ctx: Context, mode: int) -> None:

@@ -110,6 +110,9 @@ extern "C" tasq_status tasq_linear_forward_noalloc(const void* x, int64_t M, int
   a.s_x = s_x;
   a.n = hadamard_n;
   a.sx_factor = static_cast<float>(1.0 / (127.0 * std::sqrt(static_cast<double>(hadamard_n))));
+  a.status = status;
+  a.wait_limit_ns = 1000000000ull;
+  a.num_sms = num_sms;
   if ((e = tasq::launch_prologue(a, s)) != cudaSuccess) return tasq::fail_cuda(e, "prologue launch");
 
   CUtensorMap tw, tx, ty;

@@ -7,28 +7,35 @@
 //   s_x = a / (127 sqrt(n))              the 2^(-k/2) normalisation folded into the scale
 //                                        (HQ-DM section 2.1, "Eficiencia de Hardware")
 //
-// Work split: a CTA owns R consecutive token rows and R * L threads, L = Kp / 32. Thread i owns
-// the 32 consecutive channels [32 (i % L), 32 (i % L) + 32) of row i / L: 64 contiguous bytes in
-// (two full 32-byte sectors), 32 contiguous bytes out (one sector), all values in registers. A
-// Hadamard block of n channels is n / 32 neighbouring lanes. R is chosen on the host so that R * L
-// fills whole warps, which keeps every lane busy for any K.
+// Every thread owns 32 consecutive channels of one row, all values in registers; a Hadamard
+// block of n channels is n / 32 threads of one warp. The 32 values sit in 16 register pairs,
+// pair p = (z_p, z_(p+16)), so the butterfly stages with stride 1, 2, 4, 8 are packed FP32x2 add /
+// fma (two independent IEEE round-to-nearest operations each), the stride-16 stage runs inside
+// each pair, and the stride-32 (and, for n = 128, stride-64) stage pairs the thread with the one
+// holding the partner segment through xor shuffles and one packed fma by +-1 (exact product, one
+// rounding). The stages run in increasing stride, each butterfly (a, b) -> (a + b, a - b) rounded
+// once in FP32, so the codes are the same bits as a textbook FP32 fast Walsh-Hadamard transform
+// produces. The per-row absmax is combined through a shared-memory atomicMax on the float bits
+// (all values are non-negative). No FMA contraction happens anywhere on the path.
 //
-// The 32 values sit in 16 register pairs, pair p = (z_p, z_(p+16)), so the butterfly stages with
-// stride 1, 2, 4, 8 are packed FP32x2 add / fma (two independent IEEE round-to-nearest operations
-// each), the stride-16 stage runs inside each pair, and the stride-32 (and, for n = 128,
-// stride-64) stage pairs lane i with lane i ^ 1 (and i ^ 2) through xor shuffles and one packed
-// fma by +-1 (exact product, one rounding). The stages run in increasing stride, each butterfly (a, b) -> (a + b, a - b) rounded once in FP32, so the codes
-// are the same bits as a textbook FP32 fast Walsh-Hadamard transform produces.
-// The per-row absmax is combined through a shared-memory atomicMax on the float bits (all values
-// are non-negative). No FMA contraction happens anywhere on the path.
+// Two variants compute the same bits:
+//   bulk-fed  one persistent CTA per SM; a producer warp streams blocks of rows into a ring of
+//             shared-memory stages, one 1-D bulk copy per row, so that many bytes stay in flight
+//             while up to 31 compute warps work on the stages already landed (any K % 8 == 0).
+//   direct    a CTA owns R consecutive rows and R * Kp / 32 threads that load their 64 bytes
+//             straight from global memory (two full sectors) and store 32 (one sector); it
+//             serves the weight-only launch and arguments the bulk-fed layout does not fit.
 //
 // The same launch can also truncate a layer's weights for the step (TASQ's LSB mask,
-// w AND (0xFF << k) with k = 8 - bits): CTAs past the activation rows stream the layer's INT8
-// weights once, 32 bytes per thread and load, into a masked copy that the GEMM then reads as its
-// weight operand. Masking once per forward costs 2 N Kp bytes of HBM traffic; masking inside the
-// GEMM costs a shared-memory read and write of every weight tile for every token tile.
+// w AND (0xFF << k) with k = 8 - bits) into a masked copy that the GEMM then reads as its weight
+// operand: the bulk-fed CTAs do it after their rows, the direct variant in extra CTAs. Masking once
+// per forward costs 2 N Kp bytes of HBM traffic; masking inside the GEMM costs a shared-memory
+// read and write of every weight tile for every token tile.
 #include <cuda_fp16.h>
 
+#include <mutex>
+
+#include "ptx.cuh"
 #include "tasq_internal.h"
 
 namespace tasq {
@@ -113,39 +120,115 @@ __device__ __forceinline__ float2 fma2_sign(float2 mine, float s, float2 other) 
   return *reinterpret_cast<const float2*>(&r);
 }
 
+// ------------------------------------------------------------------------------ one segment
+// The arithmetic of one thread's 32-channel segment, shared by both variants.
+
+// u[i] holds channels 2i, 2i + 1 (FP16) -> v[p] = (z_p, z_(p+16)) in FP32 (exact).
+__device__ __forceinline__ void to_pairs(const uint32_t (&u)[16], float2 (&v)[16]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    __half2 hl, hh;
+    *reinterpret_cast<uint32_t*>(&hl) = u[i];       // channels 2i, 2i + 1
+    *reinterpret_cast<uint32_t*>(&hh) = u[i + 8];   // channels 16 + 2i, 17 + 2i
+    const float2 fl = __half22float2(hl);
+    const float2 fh = __half22float2(hh);
+    v[2 * i] = make_float2(fl.x, fh.x);
+    v[2 * i + 1] = make_float2(fl.y, fh.y);
+  }
+}
+
+// The block Hadamard butterflies of one segment, strides 1, 2, ..., n / 2 in that order, each
+// (a, b) -> (a + b, a - b) rounded once in FP32. LANES = n / 32 segments per Hadamard block; the
+// partner of segment `seg` for stride 32 m (m = 1, 2) is the thread `lane_unit * m` lanes away
+// (xor), in the same warp.
+template <int LANES>
+__device__ __forceinline__ void fwht_segment(float2 (&v)[16], int seg, int lane_unit) {
+  // strides 1, 2, 4, 8: pairs p and p + h, both halves at once
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      if ((p & h) == 0) butterfly2(v[p], v[p + h]);
+    }
+  }
+  // stride 16: inside each pair
+#pragma unroll
+  for (int p = 0; p < 16; ++p) {
+    const float lo = v[p].x, hi = v[p].y;
+    v[p].x = __fadd_rn(lo, hi);
+    v[p].y = __fsub_rn(lo, hi);
+  }
+  // strides 32 (and 64): the lower segment keeps mine + other, the upper one other - mine
+#pragma unroll
+  for (int m = 1; m < LANES; m <<= 1) {
+    const float sgn = (seg & m) != 0 ? -1.0f : 1.0f;
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      float2 o;
+      o.x = __shfl_xor_sync(0xffffffffu, v[p].x, m * lane_unit);
+      o.y = __shfl_xor_sync(0xffffffffu, v[p].y, m * lane_unit);
+      v[p] = fma2_sign(v[p], sgn, o);
+    }
+  }
+}
+
+__device__ __forceinline__ float absmax_segment(const float2 (&v)[16]) {
+  float mx = 0.0f;
+#pragma unroll
+  for (int p = 0; p < 16; ++p) mx = fmaxf(mx, fmaxf(fabsf(v[p].x), fabsf(v[p].y)));
+  return mx;
+}
+
+// Codes RNE(fp32(z * inv)) of the segment; w[j] = channels 4j .. 4j + 3, lowest channel in the
+// lowest byte.
+__device__ __forceinline__ void codes_segment(float2 (&v)[16], float inv, uint32_t (&w)[8]) {
+#pragma unroll
+  for (int p = 0; p < 16; ++p) v[p] = mul2(v[p], inv);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    w[j] = pack4(code(v[4 * j].x), code(v[4 * j + 1].x), code(v[4 * j + 2].x), code(v[4 * j + 3].x));
+    w[4 + j] = pack4(code(v[4 * j].y), code(v[4 * j + 1].y), code(v[4 * j + 2].y), code(v[4 * j + 3].y));
+  }
+}
+
 constexpr int kWeightUnroll = 4;         // 32-byte loads in flight per thread in the weight pass
 constexpr int64_t kMaxWeightCtas = 592;  // four CTAs for each of a B200's 148 SMs
 
-// Weight pass of CTA `cta` of `num_ctas`: w_dst = w_src AND the step's byte mask.
-__device__ __forceinline__ void weight_pass(const PrologueArgs& a, int64_t cta, int64_t num_ctas) {
-  // the previous GEMM may still read w_dst: wait for it, then let the next kernel start its setup
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+// Weight pass over `count` cooperating threads, thread `idx` of them.
+__device__ __forceinline__ void weight_pass_threads(const PrologueArgs& a, int64_t idx, int64_t count) {
   int bits = a.bits_table[a.bits_index];
   if (bits < 1 || bits > 8) {
-    if (cta == 0 && threadIdx.x == 0) atomicOr(a.status, TASQ_DEVICE_BAD_BITS);
+    if (idx == 0) atomicOr(a.status, TASQ_DEVICE_BAD_BITS);
     bits = 8;
   }
   const uint32_t m = 0x01010101u * ((0xFFu << (8 - bits)) & 0xFFu);
   const int64_t n32 = a.w_bytes >> 5;
-  const int64_t stride = num_ctas * blockDim.x;
-  for (int64_t i0 = cta * blockDim.x + threadIdx.x; i0 < n32; i0 += kWeightUnroll * stride) {
+  for (int64_t i0 = idx; i0 < n32; i0 += kWeightUnroll * count) {
     uint32_t u[kWeightUnroll][8];
 #pragma unroll
-    for (int j = 0; j < kWeightUnroll; ++j) {
-      const int64_t i = i0 + j * stride;
-      if (i < n32) ld_32B(a.w_src + 32 * i, u[j]);
+    for (int jj = 0; jj < kWeightUnroll; ++jj) {
+      const int64_t i = i0 + jj * count;
+      if (i < n32) ld_32B(a.w_src + 32 * i, u[jj]);
     }
 #pragma unroll
-    for (int j = 0; j < kWeightUnroll; ++j) {
-      const int64_t i = i0 + j * stride;
+    for (int jj = 0; jj < kWeightUnroll; ++jj) {
+      const int64_t i = i0 + jj * count;
       if (i < n32) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) u[j][e] &= m;
-        st_32B(a.w_dst + 32 * i, u[j]);
+        for (int e = 0; e < 8; ++e) u[jj][e] &= m;
+        st_32B(a.w_dst + 32 * i, u[jj]);
       }
     }
   }
+}
+
+// Weight pass of CTA `cta` of `num_ctas` of the direct variant: w_dst = w_src AND the step's
+// byte mask.
+__device__ __forceinline__ void weight_pass(const PrologueArgs& a, int64_t cta, int64_t num_ctas) {
+  // the previous GEMM may still read w_dst: wait for it, then let the next kernel start its setup
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  weight_pass_threads(a, cta * blockDim.x + threadIdx.x, num_ctas * blockDim.x);
 }
 
 // LANES = n / 32 lanes per Hadamard block; VEC32: row starts of x and xq are 32-byte aligned.
@@ -201,64 +284,17 @@ __global__ void __launch_bounds__(kMaxThreads)
         for (int i = 0; i < 8; ++i) ug[i] = 0u;
       }
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      __half2 hl, hh;
-      *reinterpret_cast<uint32_t*>(&hl) = u[i];       // channels 2i, 2i + 1
-      *reinterpret_cast<uint32_t*>(&hh) = u[i + 8];   // channels 16 + 2i, 17 + 2i
-      const float2 fl = __half22float2(hl);
-      const float2 fh = __half22float2(hh);
-      v[2 * i] = make_float2(fl.x, fh.x);
-      v[2 * i + 1] = make_float2(fl.y, fh.y);
-    }
+    to_pairs(u, v);
   }
-
-  // strides 1, 2, 4, 8: pairs p and p + h, both halves at once
-#pragma unroll
-  for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-    for (int p = 0; p < 16; ++p) {
-      if ((p & h) == 0) butterfly2(v[p], v[p + h]);
-    }
-  }
-  // stride 16: inside each pair
-#pragma unroll
-  for (int p = 0; p < 16; ++p) {
-    const float lo = v[p].x, hi = v[p].y;
-    v[p].x = __fadd_rn(lo, hi);
-    v[p].y = __fsub_rn(lo, hi);
-  }
-  // strides 32 (and 64): the partner segment of the block sits in lane ^ m; the lower lane keeps
-  // mine + other, the upper lane other - mine
-#pragma unroll
-  for (int m = 1; m < LANES; m <<= 1) {
-    const float sgn = (seg & m) != 0 ? -1.0f : 1.0f;
-#pragma unroll
-    for (int p = 0; p < 16; ++p) {
-      float2 o;
-      o.x = __shfl_xor_sync(0xffffffffu, v[p].x, m);
-      o.y = __shfl_xor_sync(0xffffffffu, v[p].y, m);
-      v[p] = fma2_sign(v[p], sgn, o);
-    }
-  }
-
-  float mx = 0.0f;
-#pragma unroll
-  for (int p = 0; p < 16; ++p) mx = fmaxf(mx, fmaxf(fabsf(v[p].x), fabsf(v[p].y)));
+  fwht_segment<LANES>(v, seg, 1);
+  const float mx = absmax_segment(v);
   if (active) atomicMax(&row_max[r_local], __float_as_uint(mx));
   __syncthreads();
   if (!active) return;
   const float amax = __uint_as_float(row_max[r_local]);
   const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-
-#pragma unroll
-  for (int p = 0; p < 16; ++p) v[p] = mul2(v[p], inv);
   uint32_t w[8];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {   // bytes 4j .. 4j + 3 are channels 4j .. 4j + 3
-    w[j] = pack4(code(v[4 * j].x), code(v[4 * j + 1].x), code(v[4 * j + 2].x), code(v[4 * j + 3].x));
-    w[4 + j] = pack4(code(v[4 * j].y), code(v[4 * j + 1].y), code(v[4 * j + 2].y), code(v[4 * j + 3].y));
-  }
+  codes_segment(v, inv, w);
   int8_t* dst = a.xq + row * a.Kp + c0;
   if constexpr (VEC32) {
     st_32B(dst, w);
@@ -267,6 +303,223 @@ __global__ void __launch_bounds__(kMaxThreads)
     st_16B(dst + 16, w[4], w[5], w[6], w[7]);
   }
   if (seg == 0) a.s_x[row] = __fmul_rn(amax, a.sx_factor);
+}
+
+// ------------------------------------------------------------------------------ bulk-fed variant
+constexpr int kFedMaxCompute = 992;           // compute threads per CTA (one CTA per SM)
+constexpr int kFedMaxStageBytes = 50 * 1024;
+constexpr int kFedSmemBudget = 200 * 1024;    // stage ring
+constexpr int kFedMaxStages = 8;
+
+struct FedGeom {
+  int32_t RG;           // rows per group (power of two); a row's segments sit RG lanes apart
+  int32_t R;            // rows per block, a multiple of RG
+  int32_t L;            // 32-channel segments per padded row = Kp / 32
+  int32_t T;            // compute threads = R * L; RG * L is a multiple of 32
+  int32_t row_stride;   // bytes between rows in a stage: round_up(2 K, 128) + 16
+  int32_t stages;
+  int32_t stage_bytes;  // R * row_stride rounded up to 128
+  int64_t num_blocks;   // ceil(M / R)
+  int32_t vec32;        // xq rows are 32-byte aligned
+};
+
+// AND of `p` over the T compute threads, which all wait at named barrier 1 (the barrier also
+// orders their shared-memory accesses).
+__device__ __forceinline__ bool all_compute(bool p, int T) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred q, r;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "barrier.cta.red.and.pred r, 1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, r;\n\t}"
+      : "=r"(out)
+      : "r"(static_cast<uint32_t>(p)), "r"(T)
+      : "memory");
+  return out != 0;
+}
+
+// One persistent CTA per SM. Warp T / 32 streams blocks of R rows into a ring of stages, one
+// 1-D bulk copy of 2 K bytes per row (its 32 lanes issue them), rows 16 bytes apart modulo 128 so
+// that the compute threads' 16-byte reads hit distinct banks. Compute thread t owns row
+// (t / (RG L)) RG + t % RG and segment (t / RG) % L of the block: the RG threads of a warp that
+// share a segment read RG consecutive rows, and the segments of one Hadamard block sit RG (and
+// 2 RG) lanes apart.
+template <int LANES>
+__global__ void __launch_bounds__(kFedMaxCompute + 32, 1)
+    prologue_fed_kernel(const PrologueArgs a, const FedGeom geo) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const uint32_t sbase = ptx::smem_addr(smem);
+  const int S = geo.stages;
+  const int R = geo.R;
+  const int T = geo.T;
+  const uint32_t full0 = sbase + S * geo.stage_bytes;
+  const uint32_t empty0 = full0 + 8 * S;
+  unsigned int* row_max = reinterpret_cast<unsigned int*>(smem + S * geo.stage_bytes + 16 * S);   // [3][R]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(row_max + 3 * R);
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const uint64_t limit = a.wait_limit_ns;
+
+  // x may be the previous kernel's output and the previous GEMM may still read the workspace:
+  // wait for it, then let the next kernel start its setup
+  ptx::grid_dep_wait();
+  ptx::grid_dep_launch_dependents();
+
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) {
+      ptx::mbar_init(full0 + 8 * i, 1);
+      ptx::mbar_init(empty0 + 8 * i, T / 32);
+    }
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  for (int i = tid; i < 3 * R; i += blockDim.x) row_max[i] = 0u;
+  __syncthreads();
+
+  const uint32_t row_bytes = static_cast<uint32_t>(a.K) * 2u;
+  if (tid >= T) {
+    // ------------------------------------------------------------------ producer warp
+    const char* x = static_cast<const char*>(a.x);
+    uint32_t s = 0, ph = 0, issued = 0, issued_par = 0;
+    for (int64_t rb = blockIdx.x; rb < geo.num_blocks; rb += gridDim.x) {
+      bool ok = true;
+      if (lane == 0) ok = ptx::wait_bounded(empty0 + 8 * s, ph ^ 1u, limit, abort_flag);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        if (lane == 0) {
+          atomicOr(a.status, TASQ_DEVICE_TIMEOUT_PROLOGUE);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      const int64_t left = a.M - rb * R;
+      const int rows = left < R ? static_cast<int>(left) : R;
+      if (lane == 0) ptx::mbar_arrive_expect_tx(full0 + 8 * s, static_cast<uint32_t>(rows) * row_bytes);
+      __syncwarp();
+      for (int i = lane; i < rows; i += 32) {
+        ptx::bulk_load(sbase + s * geo.stage_bytes + i * geo.row_stride, x + (rb * R + i) * a.ldx * 2, row_bytes,
+                       full0 + 8 * s);
+      }
+      issued |= 1u << s;
+      issued_par = (issued_par & ~(1u << s)) | (ph << s);
+      if (++s == static_cast<uint32_t>(S)) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+    // every copy this warp issued must have landed before the CTA may exit
+    if (lane == 0) {
+      for (int i = 0; i < S; ++i) {
+        if ((issued >> i) & 1u) {
+          if (!ptx::wait_bounded(full0 + 8 * i, (issued_par >> i) & 1u, limit, nullptr))
+            atomicOr(a.status, TASQ_DEVICE_TIMEOUT_PROLOGUE);
+        }
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------------- compute threads
+  const int RG = geo.RG;
+  const int r_in = tid & (RG - 1);
+  const int q = tid / RG;
+  const int seg = q % geo.L;
+  const int rl = (q / geo.L) * RG + r_in;         // row of the block
+  const int c0 = 32 * seg;                        // first channel of the segment
+  uint32_t s = 0, ph = 0;
+  int buf = 0;
+  bool ok = true;
+  for (int64_t rb = blockIdx.x; rb < geo.num_blocks; rb += gridDim.x) {
+    const bool got = ptx::wait_bounded(full0 + 8 * s, ph, limit, abort_flag);
+    const int64_t row = rb * R + rl;
+    const bool valid = row < a.M;
+    float2 v[16];
+    {
+      uint32_t u[16];
+      const uint8_t* src = smem + s * geo.stage_bytes + rl * geo.row_stride + 2 * c0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {   // 8 channels per 16-byte chunk; K % 8 == 0
+        if (got && valid && c0 + 8 * c + 8 <= a.K) {
+          const uint4 q4 = *reinterpret_cast<const uint4*>(src + 16 * c);
+          u[4 * c] = q4.x;
+          u[4 * c + 1] = q4.y;
+          u[4 * c + 2] = q4.z;
+          u[4 * c + 3] = q4.w;
+        } else {
+          u[4 * c] = 0u;
+          u[4 * c + 1] = 0u;
+          u[4 * c + 2] = 0u;
+          u[4 * c + 3] = 0u;
+        }
+      }
+      // the stage is in registers: hand it back to the producer (one arrival per warp)
+      if (__all_sync(0xffffffffu, got) && lane == 0) ptx::mbar_arrive(empty0 + 8 * s);
+      to_pairs(u, v);
+    }
+    fwht_segment<LANES>(v, seg, RG);
+    float mx = absmax_segment(v);
+    // the lanes of this warp that hold the same row are RG apart
+    for (int off = RG; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (got && lane < RG) atomicMax(&row_max[buf * R + rl], __float_as_uint(mx));
+    if (!all_compute(got, T)) {
+      if (tid == 0) {
+        atomicOr(a.status, TASQ_DEVICE_TIMEOUT_PROLOGUE);
+        *abort_flag = 1;
+      }
+      ok = false;
+      break;
+    }
+    // the buffer of the previous block was read before the barrier just passed: clear it for
+    // the block after next
+    const int prev = buf == 0 ? 2 : buf - 1;
+    if (seg == 0) row_max[prev * R + rl] = 0u;
+    const float amax = __uint_as_float(row_max[buf * R + rl]);
+    const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    if (valid) {
+      uint32_t w[8];
+      codes_segment(v, inv, w);
+      int8_t* dst = a.xq + row * a.Kp + c0;
+      if (geo.vec32) {
+        st_32B(dst, w);
+      } else {
+        st_16B(dst, w[0], w[1], w[2], w[3]);
+        st_16B(dst + 16, w[4], w[5], w[6], w[7]);
+      }
+      if (seg == 0) a.s_x[row] = __fmul_rn(amax, a.sx_factor);
+    }
+    buf = buf == 2 ? 0 : buf + 1;
+    if (++s == static_cast<uint32_t>(S)) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+  if (ok && a.w_bytes > 0)
+    weight_pass_threads(a, static_cast<int64_t>(blockIdx.x) * T + tid, static_cast<int64_t>(gridDim.x) * T);
+}
+
+// Geometry of the bulk-fed variant for (n, K, Kp), or R = 0 when no layout fits.
+FedGeom fed_geometry(int n, int K, int Kp) {
+  FedGeom g{};
+  g.L = Kp / 32;
+  g.row_stride = static_cast<int32_t>(round_up(static_cast<size_t>(K) * 2, 128) + 16);
+  // the segments of a Hadamard block must sit in one warp: RG * (n / 32) <= 32
+  const int rg_max = n == 64 ? 16 : 8;
+  for (int rg = rg_max; rg >= 1; rg >>= 1) {
+    if ((rg * g.L) % 32 == 0 && rg * g.L <= kFedMaxCompute) {
+      g.RG = rg;
+      break;
+    }
+  }
+  if (g.RG == 0) return g;
+  int groups = kFedMaxCompute / (g.RG * g.L);
+  while (groups > 1 && static_cast<int64_t>(groups) * g.RG * g.row_stride > kFedMaxStageBytes) --groups;
+  g.R = groups * g.RG;
+  g.T = g.R * g.L;
+  g.stage_bytes = static_cast<int32_t>(round_up(static_cast<size_t>(g.R) * g.row_stride, 128));
+  g.stages = kFedSmemBudget / g.stage_bytes;
+  if (g.stages > kFedMaxStages) g.stages = kFedMaxStages;
+  if (g.stages < 2) g.R = 0;
+  return g;
 }
 
 // rows per CTA: fill whole warps (R * C a multiple of 32) with 128..512 threads where possible
@@ -288,6 +541,63 @@ int pick_rows(int C) {
 
 }  // namespace
 
+namespace {
+
+template <int LANES>
+cudaError_t launch_fed(const PrologueArgs& a, const FedGeom& geo, int grid, int smem, cudaStream_t stream) {
+  static bool configured[64] = {false};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!configured[dev]) {
+      e = cudaFuncSetAttribute(prologue_fed_kernel<LANES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               128 + kFedSmemBudget + 16 * kFedMaxStages + 12 * 1024 + 64);
+      if (e != cudaSuccess) return e;
+      configured[dev] = true;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(geo.T + 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = use_pdl() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, prologue_fed_kernel<LANES>, a, geo);
+}
+
+// The bulk-fed variant, if it applies to these arguments (returns false otherwise). In automatic
+// mode it is taken only when each CTA streams many blocks: on B200 it beats the direct variant
+// in steady state (4.4 vs 4.0 TB/s on 17776 x 12288 rows) but loses on launches of a few blocks
+// per SM, where its ring never fills (1.9 vs 2.2 TB/s on 8192 x 1152).
+constexpr int64_t kFedMinBlocksPerSm = 32;
+
+bool try_launch_fed(const PrologueArgs& a, cudaStream_t stream, cudaError_t* err) {
+  if (a.M <= 0 || a.num_sms <= 0 || a.status == nullptr) return false;
+  if (reinterpret_cast<uintptr_t>(a.x) % 16 != 0 || a.ldx % 8 != 0 || a.K % 8 != 0 ||
+      reinterpret_cast<uintptr_t>(a.xq) % 16 != 0)
+    return false;
+  FedGeom geo = fed_geometry(a.n, a.K, a.Kp);
+  if (geo.R == 0) return false;
+  geo.num_blocks = (a.M + geo.R - 1) / geo.R;
+  if (a.variant == 0 && geo.num_blocks < kFedMinBlocksPerSm * a.num_sms) return false;
+  geo.vec32 = (reinterpret_cast<uintptr_t>(a.xq) % 32 == 0) ? 1 : 0;
+  const int64_t grid = geo.num_blocks < a.num_sms ? geo.num_blocks : a.num_sms;
+  const int smem = 128 + geo.stages * geo.stage_bytes + 16 * geo.stages + 12 * geo.R + 16;
+  *err = a.n == 64 ? launch_fed<2>(a, geo, static_cast<int>(grid), smem, stream)
+                   : launch_fed<4>(a, geo, static_cast<int>(grid), smem, stream);
+  return true;
+}
+
+}  // namespace
+
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
   const bool weights = a.w_bytes > 0;
   if (a.M <= 0 && !weights) return cudaSuccess;
@@ -295,6 +605,10 @@ cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
   if (weights && (a.w_bytes % 32 != 0 || reinterpret_cast<uintptr_t>(a.w_src) % 32 != 0 ||
                   reinterpret_cast<uintptr_t>(a.w_dst) % 32 != 0 || a.bits_table == nullptr || a.status == nullptr))
     return cudaErrorInvalidValue;
+  if (a.variant != 1) {
+    cudaError_t e = cudaSuccess;
+    if (try_launch_fed(a, stream, &e)) return e;
+  }
   const int L = a.Kp / 32;
   if (L > kMaxThreads) return cudaErrorInvalidValue;
   int R = 1, threads = 256;

@@ -138,6 +138,7 @@ struct tasq_ctx {
   float sx_factor = 0.0f;
   int32_t gemm_mode = 0;   // 0 automatic, 1 one CTA per tile, 2 CTA pairs
   int32_t mask_mode = 0;   // 0 automatic, 1 mask inside the GEMM, 2 mask ahead in the prologue launch
+  int32_t prologue_mode = 0;   // 0 automatic, 1 direct-load prologue, 2 bulk-fed prologue where it fits
   // host copy of the last schedule given, used only to choose where the mask is applied: both
   // places read the device table and give the same result for every bit width, so a device table
   // that is newer or older than this copy changes no result
@@ -246,8 +247,16 @@ tasq_status run_prologue(tasq_ctx* c, int32_t layer, int32_t step, bool weights,
   a.s_x = sx;
   a.n = c->n;
   a.sx_factor = c->sx_factor;
+  a.status = c->d_status;
+  a.wait_limit_ns = c->wait_limit_ns;
+  a.num_sms = c->num_sms;
+  a.variant = c->prologue_mode;
+  g_last_error.clear();
   cudaError_t e = tasq::launch_prologue(a, s);
-  if (e != cudaSuccess) return fail_cuda(e, "prologue launch");
+  if (e != cudaSuccess) {
+    if (!g_last_error.empty()) return fail(TASQ_ERR_CUDA, "prologue launch: " + g_last_error);
+    return fail_cuda(e, "prologue launch");
+  }
   return TASQ_OK;
 }
 
@@ -574,6 +583,14 @@ tasq_status tasq_debug_set_gemm_mode(tasq_ctx* c, int32_t mode) {
   if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
   if (mode < 0 || mode > 2) return fail(TASQ_ERR_INVALID_ARG, "mode must be 0, 1 or 2");
   c->gemm_mode = mode;
+  return TASQ_OK;
+}
+
+tasq_status tasq_debug_set_prologue_mode(tasq_ctx* c, int32_t mode) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  if (mode < 0 || mode > 2) return fail(TASQ_ERR_INVALID_ARG, "mode must be 0, 1 or 2");
+  c->prologue_mode = mode;
   return TASQ_OK;
 }
 

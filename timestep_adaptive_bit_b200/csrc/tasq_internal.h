@@ -31,7 +31,13 @@ struct PrologueArgs {
   int64_t w_bytes;
   const uint8_t* bits_table;
   int32_t bits_index;
+  // Always set: receives TASQ_DEVICE_BAD_BITS and, when a bounded wait of the bulk-fed variant
+  // gives up after wait_limit_ns, TASQ_DEVICE_TIMEOUT_PROLOGUE.
   uint32_t* status;
+  uint64_t wait_limit_ns;
+  int32_t num_sms;
+  int32_t variant;    // 0: bulk-fed for long launches, else direct; 1: always direct;
+                      // 2: bulk-fed wherever its layout fits
 };
 // Launches the activation rows (M > 0) and the weight pass (w_bytes > 0) as one grid; either
 // part may be empty.
