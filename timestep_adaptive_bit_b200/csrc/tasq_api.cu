@@ -260,24 +260,26 @@ tasq_status run_prologue(tasq_ctx* c, int32_t layer, int32_t step, bool weights,
   return TASQ_OK;
 }
 
-// Which GEMM kernel finishes first: both are persistent, so the time is the number of waves of
-// tiles times the time of one tile. A CTA pair does a 256 x 256 tile on two SMs at about 1.1x the
-// per-SM rate of one CTA on a 128 x 256 tile (measured on B200 at large K); ragged edges and
-// partial last waves decide the rest.
-bool prefer_pair(int64_t M, int64_t N, int num_sms) {
+// Which GEMM kernel finishes first. Both are persistent, so time = waves of tiles x time per
+// tile. Measured on B200: at the same wave count the CTA pair (256 x 256 tiles) beats one CTA
+// per 128 x 256 tile only once each CTA runs a long mainloop (1.14x at 12 waves x 24 K blocks,
+// CogVideoX proj). With a few hundred K blocks or less per CTA it loses up to 5 % (cluster
+// set-up and the pair's exit handshake), and with more waves it loses outright.
+bool prefer_pair(int64_t M, int64_t N, int64_t num_kb, int num_sms) {
   const int64_t t1 = ((M + 255) / 256) * ((N + 127) / 128);
   const int64_t t2 = ((M + 255) / 256) * ((N + 255) / 256);
   const int64_t slots1 = num_sms, slots2 = num_sms / 2;
-  const double w1 = static_cast<double>((t1 + slots1 - 1) / slots1);
-  const double w2 = static_cast<double>((t2 + slots2 - 1) / slots2);
-  // per-SM work per wave: 128 x 256 for one CTA, 256 x 256 / 2 for a pair
-  return w2 / 1.1 < w1;
+  const int64_t w1 = (t1 + slots1 - 1) / slots1;
+  const int64_t w2 = (t2 + slots2 - 1) / slots2;
+  if (w2 < w1) return true;
+  return w2 == w1 && w1 * num_kb >= 200;
 }
 
 tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq, const float* sx, int64_t M,
                      void* y, int64_t ldy, tasq::OutKind out, bool premasked, cudaStream_t s) {
   const LayerInfo& L = c->layers[layer];
-  const bool pair = c->gemm_mode == 2 || (c->gemm_mode == 0 && prefer_pair(M, L.N, c->num_sms));
+  const int64_t num_kb = (L.Kp + tasq::kGemmBlockK - 1) / tasq::kGemmBlockK;
+  const bool pair = c->gemm_mode == 2 || (c->gemm_mode == 0 && prefer_pair(M, L.N, num_kb, c->num_sms));
   const int tile_tok = pair ? tasq::kGemmPairTile : tasq::kGemmTileTok;
   const int tile_ch = pair ? tasq::kGemmPairTile : tasq::kGemmTileCh;
   CUtensorMap tx;
