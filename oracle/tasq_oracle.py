@@ -189,3 +189,58 @@ def masked_linear(x: np.ndarray, w: np.ndarray, s_w: np.ndarray, bits: int, n: i
 # --------------------------------------------------------------------------------------------
 def bitops(M: int, N: int, K: int, w_bits: int, a_bits: int = 8) -> int:
     return int(M) * int(N) * int(K) * int(w_bits) * int(a_bits)
+
+
+# --------------------------------------------------------------------------------------------
+# next row: DMPQ-style precision predictor (6Bit-Diffusion section 2.A, "Quantizacao de
+# Precisao Mista Dinamica (DMPQ)")
+# --------------------------------------------------------------------------------------------
+# The block's transformation magnitude at the previous step is the relative L1 distance between
+# its input and output, Gamma_(t-1) = ||out - in||_1 / ||in||_1; a light predictor keeps the
+# unstable layers (large Gamma) at 8 bits and compresses the stable ones. Readings:
+#   * the predictor is a threshold tau on Gamma: bits = hi if Gamma > tau else lo;
+#   * both norms are taken over every element of the block's FP16 input and output (same shape);
+#   * ||in||_1 = 0 carries no information, so the layer stays unstable (hi);
+#   * the two L1 sums are exact (every FP16 value is an integer multiple of 2^-24), and Gamma is
+#     their quotient in IEEE double: each sum rounded once to double, then one division.
+
+def fp16_units(x: np.ndarray) -> np.ndarray:
+    """FP16 values as exact integers in units of 2^-24 (the smallest FP16 subnormal), int64."""
+    x = np.asarray(x)
+    assert x.dtype == np.float16, "DMPQ inputs are FP16"
+    assert np.all(np.isfinite(x)), "non-finite inputs are outside the method"
+    return (x.astype(np.float64) * 2.0 ** 24).astype(np.int64)   # |x| < 2^16: exact
+
+
+def _exact_sum(a: np.ndarray) -> int:
+    """Sum of non-negative int64 values as a Python integer, in int64 chunks that cannot overflow
+    (each term < 2^41, so 2^20 terms stay below 2^61)."""
+    flat = a.reshape(-1)
+    total = 0
+    for i in range(0, flat.size, 1 << 20):
+        total += int(flat[i:i + (1 << 20)].sum(dtype=np.int64))
+    return total
+
+
+def dmpq_l1_sums(x_in: np.ndarray, x_out: np.ndarray):
+    """(||out - in||_1, ||in||_1) exactly, in units of 2^-24, as Python integers."""
+    assert x_in.shape == x_out.shape
+    u_in = fp16_units(x_in)
+    u_out = fp16_units(x_out)
+    return _exact_sum(np.abs(u_out - u_in)), _exact_sum(np.abs(u_in))
+
+
+def dmpq_gamma(x_in: np.ndarray, x_out: np.ndarray) -> float:
+    """Gamma = ||out - in||_1 / ||in||_1 in IEEE double (each exact sum rounded once to double,
+    one division); +inf when ||in||_1 = 0 and the output differs, 0 when both are 0."""
+    num, den = dmpq_l1_sums(x_in, x_out)
+    if den == 0:
+        return math.inf if num > 0 else 0.0
+    return float(num) / float(den)
+
+
+def dmpq_bits(gamma: float, tau: float, bits_unstable: int, bits_stable: int, den_zero: bool = False) -> int:
+    """The predictor's decision: unstable (Gamma > tau, or no information) keeps bits_unstable."""
+    if den_zero or gamma > tau:
+        return int(bits_unstable)
+    return int(bits_stable)

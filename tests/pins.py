@@ -192,3 +192,50 @@ def check_end_to_end(linear, block_h_exact, sylvester):
         row_l1 = np.abs(s_w.astype(np.float64)[:, None] * wk).sum(1)
         bound = 0.5 * np.asarray(out["s_x"])[:, None] * row_l1[None, :]
         assert np.all(np.abs(out["y"] - real) <= bound * (1 + 1e-6) + 1e-12), "element outside rounding bound"
+
+
+# ------------------------------------------------------------------------ DMPQ predictor
+def check_dmpq(gamma_fn, bits_fn, sums_fn):
+    from fractions import Fraction
+
+    for row in _golden_rows("dmpq_examples.txt"):
+        a, b, c, g, want = (p.strip() for p in row.split("|"))
+        x_in = np.array([float(v) for v in a.split()], dtype=np.float16)
+        x_out = np.array([float(v) for v in b.split()], dtype=np.float16)
+        tau, hi, lo = float(c.split()[0]), int(c.split()[1]), int(c.split()[2])
+        gamma = gamma_fn(x_in, x_out)
+        assert gamma == float(g), f"Gamma {gamma!r}, expected {g}"
+        den_zero = sums_fn(x_in, x_out)[1] == 0
+        assert bits_fn(gamma, tau, hi, lo, den_zero) == int(want), f"bits for row {row!r}"
+    rng = np.random.default_rng(77)
+    x = (rng.standard_normal((64, 48)) * 3).astype(np.float16)
+    x[:, 5] *= 100
+    x = x.astype(np.float16)
+    # closed forms: identity, negation, zero output, exact doubling
+    assert gamma_fn(x, x) == 0.0
+    assert gamma_fn(x, -x) == 2.0
+    assert gamma_fn(x, np.zeros_like(x)) == 1.0
+    small = (x / 8).astype(np.float16)
+    assert gamma_fn(small, (small * 2).astype(np.float16)) == 1.0
+    # invariance under a common power-of-two scale (exact in FP16 away from the range ends)
+    y = (x + rng.standard_normal(x.shape).astype(np.float16)).astype(np.float16)
+    g0 = gamma_fn(small, (y / 8).astype(np.float16))
+    assert gamma_fn((small * 4).astype(np.float16), (y / 2).astype(np.float16)) == g0
+    # invariance under any permutation of the elements applied to both tensors
+    perm = rng.permutation(x.size)
+    assert gamma_fn(x.reshape(-1)[perm], y.reshape(-1)[perm]) == gamma_fn(x, y)
+    # brute force with exact rationals on small tensors (sums below 2^53: one rounding)
+    for trial in range(20):
+        n = int(rng.integers(1, 40))
+        xi = (rng.standard_normal(n) * 10 ** rng.uniform(-6, 3)).astype(np.float16)
+        xo = (xi + rng.standard_normal(n).astype(np.float16) * np.float16(0.1)).astype(np.float16)
+        num = sum(abs(Fraction(float(o)) - Fraction(float(i))) for i, o in zip(xi, xo))
+        den = sum(abs(Fraction(float(i))) for i in xi)
+        got_num, got_den = sums_fn(xi, xo)
+        assert Fraction(got_num, 1 << 24) == num and Fraction(got_den, 1 << 24) == den, "inexact L1 sums"
+        if den > 0:
+            assert gamma_fn(xi, xo) == float(num / den), "Gamma is not the correctly rounded quotient"
+    # a large tensor: the sums must not overflow (terms up to 2^41 units, 2^22 of them)
+    big = np.full(1 << 22, 65504, dtype=np.float16)
+    num, den = sums_fn(big, -big)
+    assert den == 65504 * (1 << 24) * (1 << 22) and num == 2 * den

@@ -240,3 +240,46 @@ def test_mutation_end_to_end_unmasked():
         out["y"] = oracle.dequant(oracle.int_gemm(out["q"], w), out["s_x"], s_w)
         return out
     _fails(pins.check_end_to_end, linear, oracle.block_hadamard_exact, oracle.sylvester_hadamard)
+
+
+# ---------------------------------------------------------------- DMPQ predictor
+def _g_l2(x_in, x_out):
+    a = x_in.astype(np.float64)
+    b = x_out.astype(np.float64)
+    d = np.linalg.norm(a)
+    return float(np.linalg.norm(b - a) / d) if d > 0 else (math.inf if np.any(b != a) else 0.0)
+
+
+def _g_relative_to_output(x_in, x_out):
+    return oracle.dmpq_gamma(x_out, x_in)
+
+
+def _g_no_abs(x_in, x_out):
+    a = x_in.astype(np.float64)
+    b = x_out.astype(np.float64)
+    d = float(np.abs(a).sum())
+    return float(abs((b - a).sum()) / d) if d > 0 else (math.inf if np.any(b != a) else 0.0)
+
+
+def _g_fp16_sums(x_in, x_out):
+    d = np.abs(x_in).sum(dtype=np.float16)
+    n = np.abs((x_out - x_in).astype(np.float16)).sum(dtype=np.float16)
+    return float(n) / float(d) if d > 0 else (math.inf if n > 0 else 0.0)
+
+
+def _bits_ge(gamma, tau, hi, lo, den_zero=False):
+    return hi if (den_zero or gamma >= tau) else lo
+
+
+def _bits_zero_stable(gamma, tau, hi, lo, den_zero=False):
+    return hi if gamma > tau else lo
+
+
+@pytest.mark.parametrize("gamma_fn", [_g_l2, _g_relative_to_output, _g_no_abs, _g_fp16_sums])
+def test_mutation_dmpq_gamma(gamma_fn):
+    _fails(pins.check_dmpq, gamma_fn, oracle.dmpq_bits, oracle.dmpq_l1_sums)
+
+
+@pytest.mark.parametrize("bits_fn", [_bits_ge, _bits_zero_stable])
+def test_mutation_dmpq_decision(bits_fn):
+    _fails(pins.check_dmpq, oracle.dmpq_gamma, bits_fn, oracle.dmpq_l1_sums)

@@ -86,3 +86,7 @@ def test_outputs_fit_fp16(name):
         w, s_w = workloads.weights(wl, layer)
         y = oracle.masked_linear(x, w, s_w, 8, wl.hadamard_n)["y"]
         assert np.abs(y).max() < 65504 / 4
+
+
+def test_dmpq_predictor():
+    pins.check_dmpq(oracle.dmpq_gamma, oracle.dmpq_bits, oracle.dmpq_l1_sums)
