@@ -281,6 +281,31 @@ def setup_workload(T, torch, wl, device, out_dtype, gemm_mode=0, mask_mode=0, pr
     return ctx, xs, ys
 
 
+def time_dmpq(T, torch, ctx, wl, xs, ys, stream, reps: int = 20):
+    """CUDA-event time of tasq_dmpq_update on the block's first input and last output (same
+    width). It reads both tensors once: algorithmic bytes 2 * M * D * 2."""
+    D_in = wl.block_layers[0][1]
+    D_out = wl.block_layers[-1][2]
+    if D_in != D_out or D_in % 8 != 0:
+        return None
+    M = wl.tokens
+    x_in, x_out = xs[0], ys[D_out]
+    g = torch.zeros((1,), dtype=torch.float64, device=x_in.device)
+    layers = list(range(len(wl.block_layers)))
+    for _ in range(3):
+        T.tasq_dmpq_update(ctx, x_in, D_in, x_out, D_out, M, D_in, layers, 0, 0.05, 8, 4, g, stream)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        T.tasq_dmpq_update(ctx, x_in, D_in, x_out, D_out, M, D_in, layers, 0, 0.05, 8, 4, g, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = 1e3 * e0.elapsed_time(e1) / reps
+    return {"us": us, "gbs": 4.0 * M * D_in / (us * 1e-6) / 1e9, "shape": [M, D_in], "gamma": float(g.item())}
+
+
 def run_step(T, ctx, wl, xs, ys, step, stream):
     M = wl.tokens
     per = len(wl.block_layers)
@@ -459,6 +484,9 @@ def main(argv=None):
                "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()),
                "steps": e_steps, "ms_per_step": e_ms / e_steps}
 
+    # ---- next row: the on-device DMPQ predictor on the block's first input and last output
+    dmpq = time_dmpq(T, torch, ctx, wl, xs, ys, stream)
+
     peaks, peak_kind = load_peaks()
     int8_burst = peaks["bf16_tflops"] * INT8_OVER_BF16
     int8_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * INT8_OVER_BF16
@@ -512,6 +540,10 @@ def main(argv=None):
         "device_status": status,
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "dmpq_predictor": None if dmpq is None else {
+            "bound": "hbm", "achieved": dmpq["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": dmpq["gbs"] / peaks["hbm_gbs"], "us_per_call": dmpq["us"], "shape": dmpq["shape"],
+            "gamma": dmpq["gamma"]},
     }
     print(json.dumps(line), flush=True)
     return 0 if status == 0 else 1

@@ -59,6 +59,7 @@ typedef enum {
 
 /* Limits of this implementation. */
 #define TASQ_MAX_KP 16384           /* Kp = ceil(K / n) * n must not exceed this */
+#define TASQ_DMPQ_MAX_LAYERS 32     /* table rows one tasq_dmpq_update call may write */
 
 /*
  * One linear layer y = x W^T, described for tasq_linear_create.
@@ -167,6 +168,40 @@ tasq_status tasq_debug_gemm_s32(tasq_ctx* ctx, const int8_t* xq, int64_t M, int3
                                 int32_t* acc, int64_t ld_acc, void* stream);
 tasq_status tasq_debug_gemm(tasq_ctx* ctx, const int8_t* xq, const float* s_x, int64_t M, int32_t layer,
                             int32_t step, void* y, int64_t ldy, int32_t out_dtype, void* stream);
+
+/*
+ * Copy the device schedule table [num_layers * num_steps] (row-major by layer) into bits_host
+ * (host). Stream-ordered after everything enqueued on `stream` before it; synchronises `stream`.
+ */
+tasq_status tasq_get_schedule(tasq_ctx* ctx, uint8_t* bits_host, void* stream);
+
+/*
+ * On-device precision predictor: the DMPQ rule of 6Bit-Diffusion (technical summary, section
+ * 2.A, "Quantizacao de Precisao Mista Dinamica"). The relative L1 change of a transformer block
+ * over the previous step, Gamma = ||out - in||_1 / ||in||_1, picks the bit width of the block's
+ * linears for `step`: bits[layer][step] = Gamma > tau ? bits_unstable : bits_stable for every
+ * layer in `layers`. When ||in||_1 = 0, Gamma is +inf (or 0 if the output is zero as well) and
+ * the layers take bits_unstable. The pages compress stable layers to NVFP4; here the stable
+ * width is an LSB-masked width of the same INT8 buffer.
+ *   block_in, block_out : device FP16 [M, D], the block's input and output at the previous
+ *                         step, row strides ld_in / ld_out (elements, >= D, % 8 == 0), 16-byte
+ *                         aligned; D % 8 == 0. Neither is modified.
+ *   layers              : host array [num_block_layers] (1 .. TASQ_DMPQ_MAX_LAYERS) of layer
+ *                         indices; read before the call returns.
+ *   gamma_out           : optional device double that receives Gamma.
+ * Both L1 sums are exact (integer arithmetic in units of 2^-24); Gamma is their IEEE double
+ * quotient, each sum rounded once to nearest-even. One kernel runs on `stream` (using
+ * context-owned partial sums: calls of one context must not overlap on different streams),
+ * and the table
+ * entries change in stream order: forwards enqueued later on `stream` use the new widths,
+ * with no host round trip. Returns TASQ_ERR_INVALID_ARG for bad arguments (checked on the
+ * host before anything is enqueued), including M * D so large that a per-thread 64-bit partial
+ * sum could overflow. Non-finite inputs give an undefined decision.
+ */
+tasq_status tasq_dmpq_update(tasq_ctx* ctx, const void* block_in, int64_t ld_in, const void* block_out,
+                             int64_t ld_out, int64_t M, int32_t D, const int32_t* layers,
+                             int32_t num_block_layers, int32_t step, double tau, int32_t bits_unstable,
+                             int32_t bits_stable, double* gamma_out, void* stream);
 
 /*
  * Test hook: which GEMM kernel later forwards of this context use. 0 (default) lets the library

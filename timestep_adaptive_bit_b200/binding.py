@@ -36,6 +36,7 @@ TASQ_DEVICE_TIMEOUT_PROLOGUE = 0x20
 TASQ_DEVICE_BAD_BITS = 0x100
 
 TASQ_MAX_KP = 16384
+TASQ_DMPQ_MAX_LAYERS = 32
 TASQ_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
@@ -72,6 +73,8 @@ def _load():
         "tasq_debug_stuck_wait": [P, P],
         "tasq_debug_set_gemm_mode": [P, i32],
         "tasq_debug_set_mask_mode": [P, i32],
+        "tasq_get_schedule": [P, P, P],
+        "tasq_dmpq_update": [P, P, i64, P, i64, i64, i32, P, i32, i32, ctypes.c_double, i32, i32, P, P],
         "tasq_debug_set_prologue_mode": [P, i32],
         "tasq_trace_enable": [P, i32],
         "tasq_linear_forward_noalloc": [P, i64, i64, i32, P, P, i32, i32, i32, P, i64, i32, P, P],
@@ -125,9 +128,10 @@ def _stream(s) -> int | None:
 class Context:
     """Opaque tasq_ctx* handle (frees itself when garbage-collected if not destroyed)."""
 
-    def __init__(self, handle: int, layers: Sequence[tuple]):
+    def __init__(self, handle: int, layers: Sequence[tuple], num_steps: int = 1):
         self.handle = handle
         self.layers = [(int(N), int(K)) for N, K, *_ in layers]
+        self.num_steps = int(num_steps)
 
     @property
     def _as_parameter_(self):
@@ -161,7 +165,7 @@ def tasq_linear_create(layers: Iterable[tuple], num_steps: int, hadamard_n: int,
     _check(lib.tasq_linear_create(ctypes.byref(h), arr, len(layers), int(num_steps), int(hadamard_n),
                                   int(max_tokens), int(out_dtype), _stream(stream)))
     del keep
-    return Context(h.value, layers)
+    return Context(h.value, layers, num_steps)
 
 
 def tasq_set_schedule(ctx: Context, bits, stream=None) -> None:
@@ -172,6 +176,22 @@ def tasq_set_schedule(ctx: Context, bits, stream=None) -> None:
 def tasq_linear_forward(ctx: Context, x, M: int, ldx: int, layer: int, step: int, y, ldy: int, stream=None) -> None:
     _check(lib.tasq_linear_forward(ctx, _ptr(x), int(M), int(ldx), int(layer), int(step), _ptr(y), int(ldy),
                                    _stream(stream)))
+
+
+def tasq_get_schedule(ctx: Context, stream=None) -> np.ndarray:
+    """The device schedule table as a host uint8 array [num_layers, num_steps]."""
+    n = (len(ctx.layers), ctx.num_steps)
+    out = np.empty(n, dtype=np.uint8)
+    _check(lib.tasq_get_schedule(ctx, out.ctypes.data, _stream(stream)))
+    return out
+
+
+def tasq_dmpq_update(ctx: Context, block_in, ld_in: int, block_out, ld_out: int, M: int, D: int, layers, step: int,
+                     tau: float, bits_unstable: int, bits_stable: int, gamma_out=None, stream=None) -> None:
+    idx = np.ascontiguousarray(np.asarray(list(layers), dtype=np.int32))
+    _check(lib.tasq_dmpq_update(ctx, _ptr(block_in), int(ld_in), _ptr(block_out), int(ld_out), int(M), int(D),
+                                idx.ctypes.data, int(idx.size), int(step), float(tau), int(bits_unstable),
+                                int(bits_stable), _ptr(gamma_out), _stream(stream)))
 
 
 def tasq_linear_destroy(ctx: Context) -> None:

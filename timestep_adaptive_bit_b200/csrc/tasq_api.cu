@@ -134,6 +134,8 @@ struct tasq_ctx {
   int8_t* d_xq = nullptr;
   float* d_sx = nullptr;
   uint32_t* d_status = nullptr;
+  uint64_t* d_dmpq = nullptr;          // per-CTA partial sums of the DMPQ predictor
+  unsigned int* d_dmpq_arrived = nullptr;   // its CTA arrival counter (zero between calls)
   uint64_t wait_limit_ns = 1000000000ull;
   float sx_factor = 0.0f;
   int32_t gemm_mode = 0;   // 0 automatic, 1 one CTA per tile, 2 CTA pairs
@@ -163,6 +165,8 @@ void free_ctx(tasq_ctx* c) {
   cudaFree(c->d_xq);
   cudaFree(c->d_sx);
   cudaFree(c->d_status);
+  cudaFree(c->d_dmpq);
+  cudaFree(c->d_dmpq_arrived);
   for (auto& t : c->trace) {
     cudaEventDestroy(t.e0);
     cudaEventDestroy(t.e1);
@@ -403,6 +407,12 @@ tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, in
   if ((e = cudaMalloc(&c->d_sx, static_cast<size_t>(max_tokens) * sizeof(float))) != cudaSuccess)
     return bail(e, "cudaMalloc(workspace scales)");
   if ((e = cudaMalloc(&c->d_status, sizeof(uint32_t))) != cudaSuccess) return bail(e, "cudaMalloc(status)");
+  if ((e = cudaMalloc(&c->d_dmpq, 4 * sizeof(uint64_t) * static_cast<size_t>(c->num_sms) * tasq::kDmpqCtasPerSm)) !=
+      cudaSuccess)
+    return bail(e, "cudaMalloc(predictor partial sums)");
+  if ((e = cudaMalloc(&c->d_dmpq_arrived, sizeof(unsigned int))) != cudaSuccess) return bail(e, "cudaMalloc(counter)");
+  if ((e = cudaMemsetAsync(c->d_dmpq_arrived, 0, sizeof(unsigned int), s)) != cudaSuccess)
+    return bail(e, "cudaMemsetAsync(counter)");
 
   if ((e = cudaMemsetAsync(c->d_bits, 8, table, s)) != cudaSuccess) return bail(e, "cudaMemsetAsync(schedule)");
   c->bits_host.assign(table, 8);
@@ -578,6 +588,68 @@ tasq_status tasq_debug_gemm(tasq_ctx* c, const int8_t* xq, const float* s_x, int
   if (M == 0) return TASQ_OK;
   const tasq::OutKind out = out_dtype == TASQ_OUT_BF16 ? tasq::OutKind::BF16 : tasq::OutKind::F16;
   return debug_gemm(c, layer, step, xq, s_x, M, y, ldy, out, static_cast<cudaStream_t>(stream));
+}
+
+tasq_status tasq_get_schedule(tasq_ctx* c, uint8_t* bits_host, void* stream) {
+  g_last_error.clear();
+  if (c == nullptr || bits_host == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx or bits is NULL");
+  tasq_status st = check_device(c);
+  if (st != TASQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t table = static_cast<size_t>(c->num_layers) * c->num_steps;
+  cudaError_t e = cudaMemcpyAsync(bits_host, c->d_bits, table, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail_cuda(e, "read of schedule");
+  return TASQ_OK;
+}
+
+tasq_status tasq_dmpq_update(tasq_ctx* c, const void* block_in, int64_t ld_in, const void* block_out, int64_t ld_out,
+                             int64_t M, int32_t D, const int32_t* layers, int32_t num_block_layers, int32_t step,
+                             double tau, int32_t bits_unstable, int32_t bits_stable, double* gamma_out, void* stream) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  tasq_status st;
+  if ((st = check_step(c, step)) != TASQ_OK) return st;
+  if (layers == nullptr || num_block_layers < 1 || num_block_layers > TASQ_DMPQ_MAX_LAYERS)
+    return fail(TASQ_ERR_INVALID_ARG, "need 1 to TASQ_DMPQ_MAX_LAYERS layer indices");
+  for (int32_t i = 0; i < num_block_layers; ++i)
+    if ((st = check_layer(c, layers[i])) != TASQ_OK) return st;
+  if (bits_unstable < 1 || bits_unstable > 8 || bits_stable < 1 || bits_stable > 8)
+    return fail(TASQ_ERR_INVALID_ARG, "bit widths must be in [1, 8]");
+  if (!(tau == tau)) return fail(TASQ_ERR_INVALID_ARG, "tau is NaN");
+  if (M < 0 || M > 0x7fffffffLL) return fail(TASQ_ERR_INVALID_ARG, "M out of range");
+  if (D < 8 || D % 8 != 0) return fail(TASQ_ERR_INVALID_ARG, "D must be a positive multiple of 8");
+  if ((st = check_rows(block_in, ld_in, D, "block_in")) != TASQ_OK) return st;
+  if ((st = check_rows(block_out, ld_out, D, "block_out")) != TASQ_OK) return st;
+  if (gamma_out != nullptr && reinterpret_cast<uintptr_t>(gamma_out) % 8 != 0)
+    return fail(TASQ_ERR_INVALID_ARG, "gamma_out must be 8-byte aligned");
+  // every thread of the reduction adds at most 2^21 terms below 2^41 units: no 64-bit overflow
+  const int ctas = tasq::dmpq_partial_ctas(M, D, c->num_sms);
+  const int64_t per_thread = (M * D + static_cast<int64_t>(ctas) * 256 - 1) / (static_cast<int64_t>(ctas) * 256);
+  if (per_thread > (1LL << 21)) return fail(TASQ_ERR_INVALID_ARG, "M * D too large for exact 64-bit partial sums");
+  if ((st = check_device(c)) != TASQ_OK) return st;
+  tasq::DmpqArgs a{};
+  a.in = block_in;
+  a.out = block_out;
+  a.ld_in = ld_in;
+  a.ld_out = ld_out;
+  a.M = M;
+  a.D = D;
+  a.tau = tau;
+  a.bits_unstable = bits_unstable;
+  a.bits_stable = bits_stable;
+  a.table = c->d_bits;
+  a.num_entries = num_block_layers;
+  for (int32_t i = 0; i < num_block_layers; ++i) a.entries[i] = layers[i] * c->num_steps + step;
+  a.gamma_out = gamma_out;
+  cudaError_t e = tasq::launch_dmpq(a, c->d_dmpq, c->d_dmpq_arrived, c->num_sms, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "predictor launch");
+  // the host copy of the table only steers where the mask is applied: take the narrower width,
+  // so that a dropped bit is masked once ahead of the GEMM whichever way the device decides
+  const uint8_t hint = static_cast<uint8_t>(bits_unstable < bits_stable ? bits_unstable : bits_stable);
+  for (int32_t i = 0; i < num_block_layers; ++i)
+    c->bits_host[static_cast<size_t>(layers[i]) * c->num_steps + step] = hint;
+  return TASQ_OK;
 }
 
 tasq_status tasq_debug_set_gemm_mode(tasq_ctx* c, int32_t mode) {

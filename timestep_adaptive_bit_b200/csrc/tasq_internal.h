@@ -45,6 +45,29 @@ cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream);
 
 enum class OutKind : int { F16 = 0, BF16 = 1, S32 = 2 };
 
+// DMPQ precision predictor: Gamma = ||out - in||_1 / ||in||_1 over FP16 [M, D] (D % 8 == 0,
+// rows 16-byte aligned), then table[entries[i]] = Gamma > tau ? bits_unstable : bits_stable.
+constexpr int kDmpqMaxEntries = 32;
+constexpr int kDmpqCtasPerSm = 4;
+struct DmpqArgs {
+  const void* in;
+  const void* out;
+  int64_t ld_in, ld_out;   // row strides in elements
+  int64_t M;
+  int32_t D;
+  double tau;
+  int32_t bits_unstable, bits_stable;
+  uint8_t* table;
+  int32_t num_entries;
+  int32_t entries[kDmpqMaxEntries];   // indices into the schedule table
+  double* gamma_out;                  // optional
+};
+int dmpq_partial_ctas(int64_t M, int32_t D, int num_sms);
+// One launch on `stream`; `partial` holds 4 * dmpq_partial_ctas(...) uint64 values, and
+// `arrived` is a zeroed counter that the launch leaves zeroed again.
+cudaError_t launch_dmpq(const DmpqArgs& a, uint64_t* partial, unsigned int* arrived, int num_sms,
+                        cudaStream_t stream);
+
 // Masked INT8 GEMM: y[m, c] = sum_k xq[m, k] * mask(w[c, k]) (* s_x[m] * s_w[c]).
 struct GemmArgs {
   int32_t M;
