@@ -63,6 +63,8 @@ def parse_args(argv=None):
                    help="GEMM kernel: 0 automatic, 1 one CTA per tile, 2 CTA pairs")
     p.add_argument("--mask-mode", type=int, default=0, choices=[0, 1, 2],
                    help="LSB mask: 0 automatic, 1 inside the GEMM on every tile, 2 once ahead in the prologue launch")
+    p.add_argument("--gemm-shape", default=None,
+                   help="M,N,K: time the GEMM alone on given codes (one JSON line) and exit")
     p.add_argument("--prologue-mode", type=int, default=0, choices=[0, 1, 2],
                    help="prologue kernel: 0 automatic, 1 direct loads, 2 bulk-fed ring where it fits")
     return p.parse_args(argv)
@@ -341,6 +343,42 @@ def profile_case(args):
     return 0 if st == 0 else 1
 
 
+def gemm_shape(args):
+    """CUDA-event time of the masked GEMM alone (tasq_debug_gemm on given codes) at one shape,
+    back to back, for kernel-tuning experiments."""
+    import torch
+    import timestep_adaptive_bit_b200 as T
+    M, N, K = (int(v) for v in args.gemm_shape.split(","))
+    dev = torch.device("cuda:0")
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    w = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev, generator=g)
+    s_w = torch.rand((N,), device=dev, generator=g) * 0.01 + 0.001
+    q = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev, generator=g)
+    s_x = torch.rand((M,), device=dev, generator=g) + 0.5
+    y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    s = torch.cuda.current_stream()
+    ctx = T.tasq_linear_create([(N, K, w, s_w)], 1, 64, M, T.TASQ_OUT_F16, s)
+    T.tasq_debug_set_gemm_mode(ctx, args.gemm_mode)
+    for _ in range(3):
+        T.tasq_debug_gemm(ctx, q, s_x, M, 0, 0, y, N, T.TASQ_OUT_F16, s)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(args.reps):
+        T.tasq_debug_gemm(ctx, q, s_x, M, 0, 0, y, N, T.TASQ_OUT_F16, s)
+    e1.record(s)
+    torch.cuda.synchronize()
+    us = 1e3 * e0.elapsed_time(e1) / args.reps
+    peaks, _ = load_peaks()
+    tops = 2.0 * M * N * K / (us * 1e-6) / 1e12
+    print(json.dumps({"gemm_shape": [M, N, K], "gemm_mode": args.gemm_mode, "us": us, "tops": tops,
+                      "frac_int8_burst": tops / (peaks["bf16_tflops"] * INT8_OVER_BF16),
+                      "device_status": T.tasq_get_device_status(ctx)}), flush=True)
+    return 0
+
+
 def sweep_bits(args):
     """Per-bit-width timing of one layer at full size (CUDA-event trace of each kernel)."""
     import torch
@@ -404,6 +442,8 @@ def main(argv=None):
         return profile_case(args)
     if args.sweep_bits:
         return sweep_bits(args)
+    if args.gemm_shape:
+        return gemm_shape(args)
 
     dist = None
     if world > 1:
