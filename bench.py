@@ -309,11 +309,26 @@ def time_dmpq(T, torch, ctx, wl, xs, ys, stream, reps: int = 20):
 
 
 def run_step(T, ctx, wl, xs, ys, step, stream):
+    """Every linear of every block once. Linears that read the same input (q, k, v of SDXL) run
+    as one group: one prologue, one GEMM each."""
     M = wl.tokens
     per = len(wl.block_layers)
-    for l in range(wl.num_layers):
-        _, K, N = wl.block_layers[l % per]
-        T.tasq_linear_forward(ctx, xs[l], M, K, l, step, ys[N], N, stream)
+    plan = wl.forward_plan()
+    for b in range(wl.blocks):
+        for group in plan:
+            l0 = b * per + group[0]
+            _, K, N = wl.block_layers[group[0]]
+            if len(group) == 1:
+                T.tasq_linear_forward(ctx, xs[l0], M, K, l0, step, ys[N], N, stream)
+            else:
+                Ns = [wl.block_layers[j][2] for j in group]
+                T.tasq_linear_forward_group(ctx, xs[l0], M, K, [b * per + j for j in group], step,
+                                            [ys[n] for n in Ns], Ns, stream)
+
+
+def launches_per_step(wl) -> int:
+    """Kernels one step launches: a prologue per input, a GEMM per linear."""
+    return wl.blocks * (len(wl.forward_plan()) + len(wl.block_layers))
 
 
 def profile_case(args):
@@ -576,7 +591,7 @@ def main(argv=None):
                          f"({traced_ms / trace_steps:.3f} ms per step with the events); the timed steps run "
                          "without them",
         "clocks": clocks,
-        "gpu_launches": 2 * args.steps * L,
+        "gpu_launches": args.steps * launches_per_step(wl),
         "device_status": status,
         "cpu_baseline": cpu,
         "e2e": e2e,

@@ -60,6 +60,7 @@ typedef enum {
 /* Limits of this implementation. */
 #define TASQ_MAX_KP 16384           /* Kp = ceil(K / n) * n must not exceed this */
 #define TASQ_DMPQ_MAX_LAYERS 32     /* table rows one tasq_dmpq_update call may write */
+#define TASQ_GROUP_MAX 4            /* layers one tasq_linear_forward_group call may run */
 
 /*
  * One linear layer y = x W^T, described for tasq_linear_create.
@@ -83,8 +84,8 @@ typedef struct tasq_ctx tasq_ctx;
 /*
  * Create a context owning one shared weight buffer for `num_layers` layers, a device schedule
  * table bits[num_layers][num_steps] (every entry initialised to 8 = full precision), an
- * activation workspace for up to `max_tokens` tokens, and a transient buffer for one layer's
- * masked weights (the largest N x Kp of the layers).
+ * activation workspace for up to `max_tokens` tokens, and a transient buffer for masked
+ * weights: min(num_layers, TASQ_GROUP_MAX) slots of the largest N x Kp of the layers.
  *   out         : receives the context; *out is set to NULL on failure.
  *   layers      : host array [num_layers] of layer descriptors.
  *   hadamard_n  : block size of the Hadamard transform along K, 64 or 128.
@@ -127,6 +128,23 @@ tasq_status tasq_set_schedule(tasq_ctx* ctx, const uint8_t* bits_host, void* str
  */
 tasq_status tasq_linear_forward(tasq_ctx* ctx, const void* x, int64_t M, int64_t ldx, int32_t layer,
                                 int32_t step, void* y, int64_t ldy, void* stream);
+
+/*
+ * Several linears on one input: one prologue (block Hadamard + INT8 codes of x, computed once)
+ * feeds one GEMM per layer, e.g. separate q, k and v projections of the same hidden states.
+ * Output i is computed exactly as tasq_linear_forward(ctx, x, M, ldx, layers[i], step, ys[i],
+ * ldys[i], stream) would compute it.
+ *   layers : host array [count] of layer indices sharing the same K, 1 <= count <=
+ *            min(num_layers, TASQ_GROUP_MAX).
+ *   ys     : host array [count] of device output pointers; ldys : host array [count] of their
+ *            row strides (elements, >= N of the layer, % 8 == 0).
+ * The prologue launch masks the weights of every member whose step drops bits into its own slot
+ * of the context's masked-weight buffer, which holds min(num_layers, TASQ_GROUP_MAX) slots. The
+ * same overlap rule as tasq_linear_forward applies.
+ */
+tasq_status tasq_linear_forward_group(tasq_ctx* ctx, const void* x, int64_t M, int64_t ldx,
+                                      const int32_t* layers, int32_t count, int32_t step, void* const* ys,
+                                      const int64_t* ldys, void* stream);
 
 /* Free every device allocation of the context (synchronises the device first). NULL is a no-op. */
 tasq_status tasq_linear_destroy(tasq_ctx* ctx);

@@ -237,6 +237,49 @@ def test_forward_bulk_fed_prologue_with_weight_pass(T, n, K, N, M):
     assert T.tasq_get_device_status(ctx) == 0
 
 
+@pytest.mark.parametrize("mask", [0, 1, 2])
+def test_group_forward_shares_one_prologue(T, mask):
+    """q, k and v of one input through tasq_linear_forward_group: each output equals the oracle
+    linear of its own layer at its own bit width (8, 5 and 3 here, so members mix the stored and
+    the masked-ahead weights)."""
+    rng = np.random.default_rng(31)
+    n, K, M = 64, 1280, 700
+    shapes = [1280, 640, 2000]
+    layers = []
+    for N in shapes:
+        w = rng.integers(-128, 128, size=(N, K)).astype(np.int8)
+        s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+        layers.append((N, K, w, s_w))
+    layers.append((512, 640, rng.integers(-127, 128, size=(512, 640)).astype(np.int8), np.ones(512, np.float32)))
+    ctx = _ctx(T, layers, 2, n, M)
+    T.tasq_debug_set_mask_mode(ctx, mask)
+    sched = np.array([[8, 8], [5, 8], [3, 8], [8, 8]], np.uint8)
+    T.tasq_set_schedule(ctx, sched, _stream())
+    x = _acts(rng, M, K)
+    xd = _dev(x)
+    ldys = [N + 8 for N in shapes]
+    ys = [torch.full((M, ld), float("nan"), dtype=torch.float16, device="cuda") for ld in ldys]
+    T.tasq_linear_forward_group(ctx, xd, M, K, [0, 1, 2], 0, ys, ldys, _stream())
+    torch.cuda.synchronize()
+    for (N, _, w, s_w), y, bits in zip(layers, ys, (8, 5, 3)):
+        got_all = y.float().cpu().numpy()
+        assert np.isnan(got_all[:, N:]).all(), "write past column N"
+        got = got_all[:, :N].astype(np.float64)
+        ref = oracle.masked_linear(x, w, s_w, bits, n)["y"]
+        assert np.all(np.abs(got - ref) <= F16_REL * np.abs(ref) + ABS_TINY), f"layer with bits={bits}"
+    assert T.tasq_get_device_status(ctx) == 0
+
+    def err(*a):
+        with pytest.raises(T.TasqError) as ei:
+            T.tasq_linear_forward_group(ctx, *a)
+        return ei.value.status
+
+    y0 = ys[0]
+    assert err(xd, M, K, [0, 3], 0, [y0, y0], [ldys[0], ldys[0]], _stream()) == T.TASQ_ERR_INVALID_ARG  # K differs
+    assert err(xd, M, K, [0, 1, 2, 0, 1], 0, [y0] * 5, [2008] * 5, _stream()) == T.TASQ_ERR_INVALID_ARG  # > 4
+    assert err(xd, M, K, [0, 1], 2, [y0, y0], [ldys[0], 2008], _stream()) == T.TASQ_ERR_INVALID_ARG      # step
+
+
 def test_schedule_is_stream_ordered(T):
     """A schedule change between two forwards on one stream affects only the later forward, and
     the weights are never rewritten (the same buffer serves both)."""

@@ -37,6 +37,7 @@ TASQ_DEVICE_BAD_BITS = 0x100
 
 TASQ_MAX_KP = 16384
 TASQ_DMPQ_MAX_LAYERS = 32
+TASQ_GROUP_MAX = 4
 TASQ_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
@@ -74,6 +75,7 @@ def _load():
         "tasq_debug_set_gemm_mode": [P, i32],
         "tasq_debug_set_mask_mode": [P, i32],
         "tasq_get_schedule": [P, P, P],
+        "tasq_linear_forward_group": [P, P, i64, i64, P, i32, i32, P, P, P],
         "tasq_dmpq_update": [P, P, i64, P, i64, i64, i32, P, i32, i32, ctypes.c_double, i32, i32, P, P],
         "tasq_debug_set_prologue_mode": [P, i32],
         "tasq_trace_enable": [P, i32],
@@ -176,6 +178,16 @@ def tasq_set_schedule(ctx: Context, bits, stream=None) -> None:
 def tasq_linear_forward(ctx: Context, x, M: int, ldx: int, layer: int, step: int, y, ldy: int, stream=None) -> None:
     _check(lib.tasq_linear_forward(ctx, _ptr(x), int(M), int(ldx), int(layer), int(step), _ptr(y), int(ldy),
                                    _stream(stream)))
+
+
+def tasq_linear_forward_group(ctx: Context, x, M: int, ldx: int, layers, step: int, ys, ldys, stream=None) -> None:
+    idx = np.ascontiguousarray(np.asarray(list(layers), dtype=np.int32))
+    ptrs = (ctypes.c_void_p * len(ys))(*[_ptr(y) for y in ys])
+    lds = np.ascontiguousarray(np.asarray(list(ldys), dtype=np.int64))
+    if not (idx.size == len(ys) == lds.size):
+        raise ValueError("layers, ys and ldys must have the same length")
+    _check(lib.tasq_linear_forward_group(ctx, _ptr(x), int(M), int(ldx), idx.ctypes.data, int(idx.size), int(step),
+                                         ctypes.cast(ptrs, ctypes.c_void_p), lds.ctypes.data, _stream(stream)))
 
 
 def tasq_get_schedule(ctx: Context, stream=None) -> np.ndarray:

@@ -196,27 +196,30 @@ constexpr int64_t kMaxWeightCtas = 592;  // four CTAs for each of a B200's 148 S
 
 // Weight pass over `count` cooperating threads, thread `idx` of them.
 __device__ __forceinline__ void weight_pass_threads(const PrologueArgs& a, int64_t idx, int64_t count) {
-  int bits = a.bits_table[a.bits_index];
-  if (bits < 1 || bits > 8) {
-    if (idx == 0) atomicOr(a.status, TASQ_DEVICE_BAD_BITS);
-    bits = 8;
-  }
-  const uint32_t m = 0x01010101u * ((0xFFu << (8 - bits)) & 0xFFu);
-  const int64_t n32 = a.w_bytes >> 5;
-  for (int64_t i0 = idx; i0 < n32; i0 += kWeightUnroll * count) {
-    uint32_t u[kWeightUnroll][8];
-#pragma unroll
-    for (int jj = 0; jj < kWeightUnroll; ++jj) {
-      const int64_t i = i0 + jj * count;
-      if (i < n32) ld_32B(a.w_src + 32 * i, u[jj]);
+  for (int seg = 0; seg < a.num_w; ++seg) {
+    const PrologueArgs::WeightSegment& ws = a.w[seg];
+    int bits = a.bits_table[ws.bits_index];
+    if (bits < 1 || bits > 8) {
+      if (idx == 0) atomicOr(a.status, TASQ_DEVICE_BAD_BITS);
+      bits = 8;
     }
+    const uint32_t m = 0x01010101u * ((0xFFu << (8 - bits)) & 0xFFu);
+    const int64_t n32 = ws.bytes >> 5;
+    for (int64_t i0 = idx; i0 < n32; i0 += kWeightUnroll * count) {
+      uint32_t u[kWeightUnroll][8];
 #pragma unroll
-    for (int jj = 0; jj < kWeightUnroll; ++jj) {
-      const int64_t i = i0 + jj * count;
-      if (i < n32) {
+      for (int jj = 0; jj < kWeightUnroll; ++jj) {
+        const int64_t i = i0 + jj * count;
+        if (i < n32) ld_32B(ws.src + 32 * i, u[jj]);
+      }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) u[jj][e] &= m;
-        st_32B(a.w_dst + 32 * i, u[jj]);
+      for (int jj = 0; jj < kWeightUnroll; ++jj) {
+        const int64_t i = i0 + jj * count;
+        if (i < n32) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) u[jj][e] &= m;
+          st_32B(ws.dst + 32 * i, u[jj]);
+        }
       }
     }
   }
@@ -493,7 +496,7 @@ __global__ void __launch_bounds__(kFedMaxCompute + 32, 1)
       ph ^= 1u;
     }
   }
-  if (ok && a.w_bytes > 0)
+  if (ok && a.num_w > 0)
     weight_pass_threads(a, static_cast<int64_t>(blockIdx.x) * T + tid, static_cast<int64_t>(gridDim.x) * T);
 }
 
@@ -599,12 +602,19 @@ bool try_launch_fed(const PrologueArgs& a, cudaStream_t stream, cudaError_t* err
 }  // namespace
 
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
-  const bool weights = a.w_bytes > 0;
+  const bool weights = a.num_w > 0;
   if (a.M <= 0 && !weights) return cudaSuccess;
   if (a.Kp % a.n != 0 || (a.n != 64 && a.n != 128)) return cudaErrorInvalidValue;
-  if (weights && (a.w_bytes % 32 != 0 || reinterpret_cast<uintptr_t>(a.w_src) % 32 != 0 ||
-                  reinterpret_cast<uintptr_t>(a.w_dst) % 32 != 0 || a.bits_table == nullptr || a.status == nullptr))
-    return cudaErrorInvalidValue;
+  if (a.num_w < 0 || a.num_w > kMaxWeightSegments) return cudaErrorInvalidValue;
+  int64_t w_bytes = 0;
+  for (int i = 0; i < a.num_w; ++i) {
+    const PrologueArgs::WeightSegment& ws = a.w[i];
+    if (ws.bytes % 32 != 0 || reinterpret_cast<uintptr_t>(ws.src) % 32 != 0 ||
+        reinterpret_cast<uintptr_t>(ws.dst) % 32 != 0)
+      return cudaErrorInvalidValue;
+    w_bytes += ws.bytes;
+  }
+  if (weights && (a.bits_table == nullptr || a.status == nullptr)) return cudaErrorInvalidValue;
   if (a.variant != 1) {
     cudaError_t e = cudaSuccess;
     if (try_launch_fed(a, stream, &e)) return e;
@@ -622,7 +632,7 @@ cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
   if (weights) {
     // about kWeightUnroll 32-byte loads per thread; larger layers loop
     const int64_t per_cta = static_cast<int64_t>(threads) * 32 * kWeightUnroll;
-    weight_ctas = (a.w_bytes + per_cta - 1) / per_cta;
+    weight_ctas = (w_bytes + per_cta - 1) / per_cta;
     if (weight_ctas > kMaxWeightCtas) weight_ctas = kMaxWeightCtas;
   }
   const int64_t grid = row_ctas + weight_ctas;

@@ -145,8 +145,10 @@ struct tasq_ctx {
   // places read the device table and give the same result for every bit width, so a device table
   // that is newer or older than this copy changes no result
   std::vector<uint8_t> bits_host;
-  int8_t* d_wk = nullptr;              // masked copy of one layer's weights (largest N x Kp)
-  std::vector<CUtensorMap> tmap_wk;    // per layer, over d_wk
+  int8_t* d_wk = nullptr;              // masked copies: wk_slots slots of wk_slot_bytes each
+  size_t wk_slot_bytes = 0;            // largest N x Kp, rounded up to 1024
+  int32_t wk_slots = 0;                // min(num_layers, TASQ_GROUP_MAX)
+  std::vector<CUtensorMap> tmap_wk;    // per layer, over slot 0
   // trace
   int32_t trace_cap = 0, trace_count = 0;
   std::vector<TraceRec> trace;
@@ -224,24 +226,29 @@ bool mask_ahead(const tasq_ctx* c, int32_t layer, int32_t step) {
   return c->bits_host[static_cast<size_t>(layer) * c->num_steps + step] < 8;
 }
 
-// The prologue launch's weight-pass fields for (layer, step).
-void set_weight_pass(tasq::PrologueArgs& a, const tasq_ctx* c, int32_t layer, int32_t step) {
+int8_t* wk_slot(const tasq_ctx* c, int32_t slot) { return c->d_wk + static_cast<size_t>(slot) * c->wk_slot_bytes; }
+
+// Add (layer, step) to the prologue launch's weight pass, masked into slot `slot`.
+void add_weight_pass(tasq::PrologueArgs& a, const tasq_ctx* c, int32_t layer, int32_t step, int32_t slot) {
   const LayerInfo& L = c->layers[layer];
-  a.w_src = c->d_w + L.w_off;
-  a.w_dst = c->d_wk;
-  a.w_bytes = static_cast<int64_t>(L.N) * L.Kp;
+  tasq::PrologueArgs::WeightSegment& ws = a.w[a.num_w++];
+  ws.src = c->d_w + L.w_off;
+  ws.dst = wk_slot(c, slot);
+  ws.bytes = static_cast<int64_t>(L.N) * L.Kp;
+  ws.bits_index = layer * c->num_steps + step;
   a.bits_table = c->d_bits;
-  a.bits_index = layer * c->num_steps + step;
   a.status = c->d_status;
 }
 
 // Activation prologue of (layer, step) over M rows (M may be 0), with the weight pass when
 // `weights` is set.
-tasq_status run_prologue(tasq_ctx* c, int32_t layer, int32_t step, bool weights, const void* x, int64_t M,
-                         int64_t ldx, int8_t* xq, float* sx, cudaStream_t s) {
+// `masked` lists up to kMaxWeightSegments layers whose weights the same launch masks, layer
+// masked[i] into masked-weight slot i.
+tasq_status run_prologue(tasq_ctx* c, int32_t layer, int32_t step, const std::vector<int32_t>& masked, const void* x,
+                         int64_t M, int64_t ldx, int8_t* xq, float* sx, cudaStream_t s) {
   const LayerInfo& L = c->layers[layer];
   tasq::PrologueArgs a{};
-  if (weights) set_weight_pass(a, c, layer, step);
+  for (size_t i = 0; i < masked.size(); ++i) add_weight_pass(a, c, masked[i], step, static_cast<int32_t>(i));
   a.x = x;
   a.ldx = ldx;
   a.K = L.K;
@@ -279,8 +286,9 @@ bool prefer_pair(int64_t M, int64_t N, int64_t num_kb, int num_sms) {
   return w2 == w1 && w1 * num_kb >= 200;
 }
 
+// GEMM of (layer, step). premasked: the weights come masked from masked-weight slot `slot`.
 tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq, const float* sx, int64_t M,
-                     void* y, int64_t ldy, tasq::OutKind out, bool premasked, cudaStream_t s) {
+                     void* y, int64_t ldy, tasq::OutKind out, bool premasked, cudaStream_t s, int32_t slot = 0) {
   const LayerInfo& L = c->layers[layer];
   const int64_t num_kb = (L.Kp + tasq::kGemmBlockK - 1) / tasq::kGemmBlockK;
   const bool pair = c->gemm_mode == 2 || (c->gemm_mode == 0 && prefer_pair(M, L.N, num_kb, c->num_sms));
@@ -312,7 +320,12 @@ tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq,
   g.status = c->d_status;
   g.wait_limit_ns = c->wait_limit_ns;
   g.premasked = premasked ? 1 : 0;
-  const CUtensorMap& tw = premasked ? c->tmap_wk[layer] : c->tmap_w[layer];
+  CUtensorMap tw = premasked ? c->tmap_wk[layer] : c->tmap_w[layer];
+  if (premasked && slot != 0) {
+    st = make_tmap_u8(&tw, wk_slot(c, slot), static_cast<uint64_t>(L.Kp), static_cast<uint64_t>(L.N),
+                      tasq::kGemmBlockK, tasq::kGemmTileCh);
+    if (st != TASQ_OK) return st;
+  }
   cudaError_t e = pair ? tasq::launch_masked_gemm_pair(tw, tx, ty, g, out, c->num_sms, s)
                        : tasq::launch_masked_gemm(tw, tx, ty, g, out, c->num_sms, s);
   if (e != cudaSuccess) return fail_cuda(e, "masked GEMM launch");
@@ -324,7 +337,7 @@ tasq_status debug_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* x
                        int64_t ldy, tasq::OutKind out, cudaStream_t s) {
   const bool ahead = mask_ahead(c, layer, step);
   tasq_status st;
-  if (ahead && (st = run_prologue(c, layer, step, true, nullptr, 0, 0, nullptr, nullptr, s)) != TASQ_OK) return st;
+  if (ahead && (st = run_prologue(c, layer, step, {layer}, nullptr, 0, 0, nullptr, nullptr, s)) != TASQ_OK) return st;
   return run_gemm(c, layer, step, xq, sx, M, y, ldy, out, ahead, s);
 }
 
@@ -398,7 +411,10 @@ tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, in
     return st;
   };
   if ((e = cudaMalloc(&c->d_w, w_bytes)) != cudaSuccess) return bail(e, "cudaMalloc(weights)");
-  if ((e = cudaMalloc(&c->d_wk, wk_bytes)) != cudaSuccess) return bail(e, "cudaMalloc(masked weights)");
+  c->wk_slot_bytes = round_up(wk_bytes, 1024);
+  c->wk_slots = num_layers < TASQ_GROUP_MAX ? num_layers : TASQ_GROUP_MAX;
+  if ((e = cudaMalloc(&c->d_wk, c->wk_slot_bytes * c->wk_slots)) != cudaSuccess)
+    return bail(e, "cudaMalloc(masked weights)");
   if ((e = cudaMalloc(&c->d_sw, sw_count * sizeof(float))) != cudaSuccess) return bail(e, "cudaMalloc(scales)");
   const size_t table = static_cast<size_t>(num_layers) * num_steps;
   if ((e = cudaMalloc(&c->d_bits, table)) != cudaSuccess) return bail(e, "cudaMalloc(schedule)");
@@ -481,7 +497,9 @@ tasq_status tasq_linear_forward(tasq_ctx* c, const void* x, int64_t M, int64_t l
   TraceRec* tr = c->trace_count < c->trace_cap ? &c->trace[c->trace_count] : nullptr;
   const bool ahead = mask_ahead(c, layer, step);
   if (tr) cudaEventRecord(tr->e0, s);
-  if ((st = run_prologue(c, layer, step, ahead, x, M, ldx, c->d_xq, c->d_sx, s)) != TASQ_OK) return st;
+  if ((st = run_prologue(c, layer, step, ahead ? std::vector<int32_t>{layer} : std::vector<int32_t>{}, x, M, ldx,
+                         c->d_xq, c->d_sx, s)) != TASQ_OK)
+    return st;
   if (tr) cudaEventRecord(tr->e1, s);
   const tasq::OutKind out = c->out_dtype == TASQ_OUT_BF16 ? tasq::OutKind::BF16 : tasq::OutKind::F16;
   if ((st = run_gemm(c, layer, step, c->d_xq, c->d_sx, M, y, ldy, out, ahead, s)) != TASQ_OK) return st;
@@ -489,6 +507,62 @@ tasq_status tasq_linear_forward(tasq_ctx* c, const void* x, int64_t M, int64_t l
     cudaEventRecord(tr->e2, s);
     tr->ops = 2.0 * static_cast<double>(M) * L.N * L.K;
     tr->bytes = static_cast<double>(M) * (2.0 * L.K + L.Kp + 4.0) + (ahead ? 2.0 * L.N * L.Kp : 0.0);
+    ++c->trace_count;
+  }
+  return TASQ_OK;
+}
+
+tasq_status tasq_linear_forward_group(tasq_ctx* c, const void* x, int64_t M, int64_t ldx, const int32_t* layers,
+                                      int32_t count, int32_t step, void* const* ys, const int64_t* ldys, void* stream) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  if (layers == nullptr || ys == nullptr || ldys == nullptr) return fail(TASQ_ERR_INVALID_ARG, "NULL array");
+  if (count < 1 || count > c->wk_slots)
+    return fail(TASQ_ERR_INVALID_ARG, "count must be in [1, min(num_layers, TASQ_GROUP_MAX)]");
+  tasq_status st;
+  if ((st = check_step(c, step)) != TASQ_OK) return st;
+  if ((st = check_tokens(c, M)) != TASQ_OK) return st;
+  for (int32_t i = 0; i < count; ++i) {
+    if ((st = check_layer(c, layers[i])) != TASQ_OK) return st;
+    if (c->layers[layers[i]].K != c->layers[layers[0]].K)
+      return fail(TASQ_ERR_INVALID_ARG, "the layers of a group must share K");
+    if ((st = check_rows(ys[i], ldys[i], c->layers[layers[i]].N, "y")) != TASQ_OK) return st;
+  }
+  const LayerInfo& L0 = c->layers[layers[0]];
+  if ((st = check_rows(x, ldx, L0.K, "x")) != TASQ_OK) return st;
+  if ((st = check_device(c)) != TASQ_OK) return st;
+  if (M == 0) return TASQ_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // one prologue for the shared input; it also masks, each into its own slot, the weights of
+  // every member whose step drops bits
+  std::vector<int32_t> masked;
+  std::vector<int32_t> slot_of(count, -1);
+  for (int32_t i = 0; i < count; ++i) {
+    if (mask_ahead(c, layers[i], step)) {
+      slot_of[i] = static_cast<int32_t>(masked.size());
+      masked.push_back(layers[i]);
+    }
+  }
+  TraceRec* tr = c->trace_count < c->trace_cap ? &c->trace[c->trace_count] : nullptr;
+  if (tr) cudaEventRecord(tr->e0, s);
+  if ((st = run_prologue(c, layers[0], step, masked, x, M, ldx, c->d_xq, c->d_sx, s)) != TASQ_OK) return st;
+  if (tr) cudaEventRecord(tr->e1, s);
+  const tasq::OutKind out = c->out_dtype == TASQ_OUT_BF16 ? tasq::OutKind::BF16 : tasq::OutKind::F16;
+  double ops = 0.0, wbytes = 0.0;
+  for (int32_t i = 0; i < count; ++i) {
+    const LayerInfo& L = c->layers[layers[i]];
+    const bool ahead = slot_of[i] >= 0;
+    if ((st = run_gemm(c, layers[i], step, c->d_xq, c->d_sx, M, ys[i], ldys[i], out, ahead, s,
+                       ahead ? slot_of[i] : 0)) != TASQ_OK)
+      return st;
+    ops += 2.0 * static_cast<double>(M) * L.N * L.K;
+    if (ahead) wbytes += 2.0 * L.N * L.Kp;
+  }
+  if (tr) {
+    cudaEventRecord(tr->e2, s);
+    tr->ops = ops;
+    tr->bytes = static_cast<double>(M) * (2.0 * L0.K + L0.Kp + 4.0) + wbytes;
     ++c->trace_count;
   }
   return TASQ_OK;
@@ -552,7 +626,7 @@ tasq_status tasq_debug_quantize(tasq_ctx* c, const void* x, int64_t M, int64_t l
   if (s_x == nullptr || !aligned16(s_x)) return fail(TASQ_ERR_INVALID_ARG, "s_x must be a 16-byte aligned pointer");
   if ((st = check_device(c)) != TASQ_OK) return st;
   if (M == 0) return TASQ_OK;
-  return run_prologue(c, layer, 0, false, x, M, ldx, xq, s_x, static_cast<cudaStream_t>(stream));
+  return run_prologue(c, layer, 0, {}, x, M, ldx, xq, s_x, static_cast<cudaStream_t>(stream));
 }
 
 tasq_status tasq_debug_gemm_s32(tasq_ctx* c, const int8_t* xq, int64_t M, int32_t layer, int32_t step, int32_t* acc,

@@ -12,6 +12,8 @@
 namespace tasq {
 
 // Activation prologue: block Hadamard along K, per-token absmax, RNE INT8 codes.
+constexpr int kMaxWeightSegments = 4;   // layers one prologue launch can mask (= TASQ_GROUP_MAX)
+
 struct PrologueArgs {
   const void* x;      // FP16 [M, K], row stride ldx elements
   int64_t ldx;
@@ -22,15 +24,19 @@ struct PrologueArgs {
   float* s_x;         // [M]
   int32_t n;          // 64 or 128
   float sx_factor;    // fp32(1 / (127 sqrt(n)))
-  // Optional weight pass in the same launch (w_bytes > 0): w_dst = w_src AND the byte mask
-  // 0xFF << (8 - bits), bits = bits_table[bits_index]; out-of-range bits set
-  // TASQ_DEVICE_BAD_BITS in *status and are read as 8. Both buffers 32-byte aligned, w_bytes a
+  // Optional weight pass in the same launch (num_w > 0): for each segment, dst = src AND the
+  // byte mask 0xFF << (8 - bits), bits = bits_table[bits_index]; out-of-range bits set
+  // TASQ_DEVICE_BAD_BITS in *status and are read as 8. Buffers 32-byte aligned, bytes a
   // multiple of 32.
-  const int8_t* w_src;
-  int8_t* w_dst;
-  int64_t w_bytes;
+  struct WeightSegment {
+    const int8_t* src;
+    int8_t* dst;
+    int64_t bytes;
+    int32_t bits_index;
+  };
+  int32_t num_w;
+  WeightSegment w[kMaxWeightSegments];
   const uint8_t* bits_table;
-  int32_t bits_index;
   // Always set: receives TASQ_DEVICE_BAD_BITS and, when a bounded wait of the bulk-fed variant
   // gives up after wait_limit_ns, TASQ_DEVICE_TIMEOUT_PROLOGUE.
   uint32_t* status;
@@ -39,7 +45,7 @@ struct PrologueArgs {
   int32_t variant;    // 0: bulk-fed for long launches, else direct; 1: always direct;
                       // 2: bulk-fed wherever its layout fits
 };
-// Launches the activation rows (M > 0) and the weight pass (w_bytes > 0) as one grid; either
+// Launches the activation rows (M > 0) and the weight pass (num_w > 0) as one grid; either
 // part may be empty.
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream);
 

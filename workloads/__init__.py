@@ -51,6 +51,20 @@ class Workload:
     fixed_bits: Tuple[int, ...] = ()         # per step, for schedule_kind == "fixed"
     outlier_kind: str = "scale50"            # "scale50" or "student_t3"
     outlier_frac: float = 0.005
+    # groups of block-layer indices that read the same input (one prologue feeds their GEMMs)
+    shared_input: Tuple[Tuple[int, ...], ...] = ()
+
+    def forward_plan(self) -> List[Tuple[int, ...]]:
+        """The block's linears in order, as tuples of block-layer indices sharing one input."""
+        lead = {g[0]: g for g in self.shared_input}
+        members = {j for g in self.shared_input for j in g}
+        plan = []
+        for j in range(len(self.block_layers)):
+            if j in lead:
+                plan.append(tuple(lead[j]))
+            elif j not in members:
+                plan.append((j,))
+        return plan
 
     @property
     def num_layers(self) -> int:
@@ -69,8 +83,10 @@ class Workload:
         return 2 * self.tokens * self.blocks * sum(K * N for _, K, N in self.block_layers)
 
     def prologue_bytes_per_step(self) -> int:
-        """Algorithmic bytes of the activation prologue per step: read 2K, write Kp + 4."""
-        return self.tokens * self.blocks * sum(2 * K + self.kp(K) + 4 for _, K, _ in self.block_layers)
+        """Algorithmic prologue bytes per step: 2K read + Kp codes + 4 scale per token and input
+        (linears sharing an input quantize it once)."""
+        return self.tokens * self.blocks * sum(
+            2 * K + self.kp(K) + 4 for K in (self.block_layers[g[0]][1] for g in self.forward_plan()))
 
 
 WORKLOADS = {
@@ -90,7 +106,7 @@ WORKLOADS = {
         block_layers=(("q", 1280, 1280), ("k", 1280, 1280), ("v", 1280, 1280), ("out", 1280, 1280),
                       ("ff_geglu", 1280, 10240), ("ff_out", 5120, 1280)),
         blocks=1, steps=4, hadamard_n=64, schedule_kind="fixed", fixed_bits=(8, 6, 5, 4),
-        outlier_kind="student_t3", outlier_frac=0.01),
+        outlier_kind="student_t3", outlier_frac=0.01, shared_input=((0, 1, 2),)),
     "cogvideox": Workload(
         name="cogvideox", tokens=13 * 30 * 45 + 226,
         block_layers=(("qkv", 3072, 9216), ("proj", 3072, 3072), ("fc1", 3072, 12288), ("fc2", 12288, 3072)),
