@@ -43,6 +43,7 @@ namespace {
 
 constexpr int kMaxRowsPerCta = 64;
 constexpr int kMaxThreads = 512;
+constexpr int kSmallThreads = 288;   // CTAs up to this size get 56 registers: 4 CTAs per SM
 
 __device__ __forceinline__ uint4 ld_16B(const void* p) {
   uint4 v;
@@ -236,8 +237,8 @@ __device__ __forceinline__ void weight_pass(const PrologueArgs& a, int64_t cta, 
 
 // LANES = n / 32 lanes per Hadamard block; VEC32: row starts of x and xq are 32-byte aligned.
 // CTAs [0, row_ctas) quantize activation rows, the rest run the weight pass.
-template <int LANES, bool VEC32>
-__global__ void __launch_bounds__(kMaxThreads)
+template <int LANES, bool VEC32, int MAXT, int MINB>
+__global__ void __launch_bounds__(MAXT, MINB)
     prologue_kernel(const PrologueArgs a, const int rows_per_cta, const int row_ctas) {
   if (static_cast<int>(blockIdx.x) >= row_ctas) {
     weight_pass(a, blockIdx.x - row_ctas, gridDim.x - row_ctas);
@@ -525,11 +526,11 @@ FedGeom fed_geometry(int n, int K, int Kp) {
   return g;
 }
 
-// rows per CTA: fill whole warps (R * C a multiple of 32) with 128..512 threads where possible
-int pick_rows(int C) {
+// rows per CTA: fill whole warps (R * C a multiple of 32) with 128..cap threads where possible
+int pick_rows(int C, int cap) {
   int best_r = 1;
   double best_score = -1.0;
-  for (int r = 1; r <= kMaxRowsPerCta && r * C <= kMaxThreads; ++r) {
+  for (int r = 1; r <= kMaxRowsPerCta && r * C <= cap; ++r) {
     const int t = r * C;
     const double util = static_cast<double>(t) / (((t + 31) / 32) * 32);
     double score = util;
@@ -623,8 +624,11 @@ cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
   if (L > kMaxThreads) return cudaErrorInvalidValue;
   int R = 1, threads = 256;
   int64_t row_ctas = 0;
+  // rows of up to 384 threads run in CTAs of at most 384 threads with 56 registers each, so four
+  // CTAs share an SM; longer rows take the 512-thread instance
+  const bool small = L <= kSmallThreads;
   if (a.M > 0) {
-    R = pick_rows(L);
+    R = pick_rows(L, small ? kSmallThreads : kMaxThreads);
     threads = ((R * L + 31) / 32) * 32;
     row_ctas = (a.M + R - 1) / R;
   }
@@ -649,12 +653,20 @@ cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = use_pdl() ? 1 : 0;
   const int rc = static_cast<int>(row_ctas);
-  if (a.n == 64) {
-    if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<2, true>, a, R, rc);
-    return cudaLaunchKernelEx(&cfg, prologue_kernel<2, false>, a, R, rc);
+  if (small) {
+    if (a.n == 64) {
+      if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<2, true, kSmallThreads, 4>, a, R, rc);
+      return cudaLaunchKernelEx(&cfg, prologue_kernel<2, false, kSmallThreads, 4>, a, R, rc);
+    }
+    if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<4, true, kSmallThreads, 4>, a, R, rc);
+    return cudaLaunchKernelEx(&cfg, prologue_kernel<4, false, kSmallThreads, 4>, a, R, rc);
   }
-  if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<4, true>, a, R, rc);
-  return cudaLaunchKernelEx(&cfg, prologue_kernel<4, false>, a, R, rc);
+  if (a.n == 64) {
+    if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<2, true, kMaxThreads, 1>, a, R, rc);
+    return cudaLaunchKernelEx(&cfg, prologue_kernel<2, false, kMaxThreads, 1>, a, R, rc);
+  }
+  if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<4, true, kMaxThreads, 1>, a, R, rc);
+  return cudaLaunchKernelEx(&cfg, prologue_kernel<4, false, kMaxThreads, 1>, a, R, rc);
 }
 
 }  // namespace tasq
