@@ -65,6 +65,8 @@ def parse_args(argv=None):
                    help="LSB mask: 0 automatic, 1 inside the GEMM on every tile, 2 once ahead in the prologue launch")
     p.add_argument("--gemm-shape", default=None,
                    help="M,N,K: time the GEMM alone on given codes (one JSON line) and exit")
+    p.add_argument("--graph", action="store_true",
+                   help="capture each schedule step's launches in a CUDA graph and time graph replays")
     p.add_argument("--prologue-mode", type=int, default=0, choices=[0, 1, 2],
                    help="prologue kernel: 0 automatic, 1 direct loads, 2 bulk-fed ring where it fits")
     return p.parse_args(argv)
@@ -474,6 +476,24 @@ def main(argv=None):
     for i in range(args.warmup):
         run_step(T, ctx, wl, xs, ys, i % wl.steps, stream)
     torch.cuda.synchronize()
+    graphs = {}
+    if args.graph:
+        # one graph per schedule step: the (layer, step) table indices are kernel arguments
+        for t in sorted({i % wl.steps for i in range(args.steps)}):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                run_step(T, ctx, wl, xs, ys, t, torch.cuda.current_stream())
+            graphs[t] = g
+        for i in range(args.warmup):
+            graphs[i % wl.steps].replay() if (i % wl.steps) in graphs else None
+        torch.cuda.synchronize()
+
+    def timed_step(i):
+        if graphs:
+            graphs[i % wl.steps].replay()
+        else:
+            run_step(T, ctx, wl, xs, ys, i % wl.steps, stream)
+
     sampler = ClockSampler(local_rank)
     if dist is not None:
         dist.barrier()
@@ -484,7 +504,7 @@ def main(argv=None):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(args.steps):
-        run_step(T, ctx, wl, xs, ys, i % wl.steps, stream)
+        timed_step(i)
     t1.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -571,6 +591,7 @@ def main(argv=None):
                    "hadamard_n": wl.hadamard_n,
                    "linears": [f"{n}:{K}->{N}" for n, K, N in wl.block_layers],
                    "out_dtype": args.out_dtype, "parallelism": f"replicas{world}",
+                   "launch": "cuda_graph_per_step" if args.graph else "stream",
                    "l2": "inputs larger than L2: each step reads its own activations for every (block, linear) "
                          f"({sum(x.numel() * 2 for x in xs) / 1e9:.2f} GB) and every layer's weights once"},
         "tokens_per_s_per_step": wl.tokens / (ms_per_step / 1e3) * world,

@@ -280,6 +280,37 @@ def test_group_forward_shares_one_prologue(T, mask):
     assert err(xd, M, K, [0, 1], 2, [y0, y0], [ldys[0], 2008], _stream()) == T.TASQ_ERR_INVALID_ARG      # step
 
 
+def test_forward_replays_from_a_cuda_graph(T):
+    """Forwards captured in a CUDA graph (prologue with the weight pass, then the GEMM, linked by
+    programmatic launch) replay to the same bits as the same forwards launched directly."""
+    rng = np.random.default_rng(41)
+    n, K, N, M = 64, 1152, 1152, 512
+    x = _acts(rng, M, K)
+    w = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+    ctx = _ctx(T, [(N, K, w, s_w), (N, K, w[::-1].copy(), s_w)], 2, n, M)
+    T.tasq_set_schedule(ctx, np.array([[5, 8], [8, 3]], np.uint8), _stream())
+    xd = _dev(x)
+    eager = [torch.empty((M, N), dtype=torch.float16, device="cuda") for _ in range(2)]
+    for layer in range(2):
+        T.tasq_linear_forward(ctx, xd, M, K, layer, layer, eager[layer], N, _stream())
+    torch.cuda.synchronize()
+    replay = [torch.zeros((M, N), dtype=torch.float16, device="cuda") for _ in range(2)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for layer in range(2):
+            T.tasq_linear_forward(ctx, xd, M, K, layer, layer, replay[layer], N, torch.cuda.current_stream())
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(eager, replay):
+        assert torch.equal(a, b)
+    ref = oracle.masked_linear(x, w, s_w, 5, n)["y"]
+    got = replay[0].float().cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - ref) <= F16_REL * np.abs(ref) + ABS_TINY)
+    assert T.tasq_get_device_status(ctx) == 0
+
+
 def test_schedule_is_stream_ordered(T):
     """A schedule change between two forwards on one stream affects only the later forward, and
     the weights are never rewritten (the same buffer serves both)."""
