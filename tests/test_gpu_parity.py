@@ -311,6 +311,31 @@ def test_forward_replays_from_a_cuda_graph(T):
     assert T.tasq_get_device_status(ctx) == 0
 
 
+def test_back_to_back_forwards_with_changing_token_counts(T):
+    """Back-to-back forwards on one stream whose token count changes every call, with and without
+    the weight pass, no synchronisation until the end: each forward reuses the workspace and the
+    masked-weight buffer after the one before it."""
+    rng = np.random.default_rng(55)
+    n, K, N = 64, 1152, 640
+    w = rng.integers(-128, 128, size=(N, K)).astype(np.int8)
+    s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+    Ms = [1000, 37, 1500, 256, 1, 999, 1500]
+    ctx = _ctx(T, [(N, K, w, s_w)], 2, n, max(Ms))
+    T.tasq_set_schedule(ctx, np.array([[8, 4]], np.uint8), _stream())
+    jobs = []
+    for i, M in enumerate(Ms):
+        x = _acts(rng, M, K)
+        y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+        T.tasq_linear_forward(ctx, _dev(x), M, K, 0, i % 2, y, N, _stream())
+        jobs.append((x, y, 8 if i % 2 == 0 else 4))
+    torch.cuda.synchronize()
+    for x, y, bits in jobs:
+        ref = oracle.masked_linear(x, w, s_w, bits, n)["y"]
+        got = y.float().cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(got - ref) <= F16_REL * np.abs(ref) + ABS_TINY), (x.shape[0], bits)
+    assert T.tasq_get_device_status(ctx) == 0
+
+
 def test_schedule_is_stream_ordered(T):
     """A schedule change between two forwards on one stream affects only the later forward, and
     the weights are never rewritten (the same buffer serves both)."""
