@@ -362,16 +362,6 @@ tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, in
   if (static_cast<int64_t>(num_layers) * num_steps > (1LL << 30))
     return fail(TASQ_ERR_INVALID_ARG, "schedule table too large");
 
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
-  cudaDeviceProp prop;
-  e = cudaGetDeviceProperties(&prop, dev);
-  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDeviceProperties");
-  if (prop.major != 10 || prop.minor != 0)
-    return fail(TASQ_ERR_UNSUPPORTED_ARCH, std::string("device ") + prop.name + " is sm_" + std::to_string(prop.major) +
-                                               std::to_string(prop.minor) + ", this library is built for sm_100a");
-
   std::vector<LayerInfo> info(num_layers);
   size_t w_bytes = 0, sw_count = 0, wk_bytes = 0;
   int32_t kp_max = 0;
@@ -391,6 +381,17 @@ tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, in
     sw_count = round_up(sw_count + d.N, 64);
     if (Kp > kp_max) kp_max = Kp;
   }
+
+  // every argument is checked on the host before the device is touched
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDeviceProperties");
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(TASQ_ERR_UNSUPPORTED_ARCH, std::string("device ") + prop.name + " is sm_" + std::to_string(prop.major) +
+                                               std::to_string(prop.minor) + ", this library is built for sm_100a");
 
   tasq_ctx* c = new tasq_ctx();
   c->device = dev;
