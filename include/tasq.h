@@ -223,11 +223,20 @@ tasq_status tasq_dmpq_update(tasq_ctx* ctx, const void* block_in, int64_t ld_in,
 
 /*
  * Test hook: which GEMM kernel later forwards of this context use. 0 (default) lets the library
- * choose per launch from the wave count of each kernel's tiles, 1 forces one CTA per 128 x 256
- * tile (tcgen05 cta_group::1), 2 forces CTA pairs on 256 x 256 tiles (tcgen05 cta_group::2).
- * Both compute identical results. Any other mode is TASQ_ERR_INVALID_ARG.
+ * choose per launch from the wave count of each kernel's tiles (tasq_gemm_choice), 1 forces one
+ * CTA per 128 x 256 tile (tcgen05 cta_group::1), 2 forces CTA pairs on 256 x 256 tiles (tcgen05
+ * cta_group::2). Both compute identical results. Any other mode is TASQ_ERR_INVALID_ARG.
  */
 tasq_status tasq_debug_set_gemm_mode(tasq_ctx* ctx, int32_t mode);
+
+/*
+ * Host-only query (no device, no context): whether a forward with the automatic choice runs the
+ * GEMM of M tokens and N output channels on a device with num_sms SMs on CTA pairs (*pair = 1,
+ * tiles of 256 channels x 256 tokens) or on one CTA per tile (*pair = 0, 128 x 256). The choice
+ * depends on these three numbers only. TASQ_ERR_INVALID_ARG for a NULL output, M or N <= 0, or
+ * num_sms < 2.
+ */
+tasq_status tasq_gemm_choice(int64_t M, int32_t N, int32_t num_sms, int32_t* pair);
 
 /*
  * Test hook: where later forwards (and tasq_debug_gemm / tasq_debug_gemm_s32) apply the step's

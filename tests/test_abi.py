@@ -114,3 +114,27 @@ def test_header_compiles_as_c99_and_links(tasq, tmp_path):
     assert r.returncode == 0, r.stderr
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == "OK", r.stdout + r.stderr
+
+
+def test_gemm_choice_is_host_only(tasq):
+    """The automatic GEMM kernel choice is a host function of (M, N, SM count). On the workloads'
+    shapes it picks the kernel that CUDA-event timings of both kernels on a B200 (148 SMs) found
+    faster (or level): CTA pairs for PixArt-Sigma fc1, SDXL ff1 and the CogVideoX linears, one CTA
+    per tile elsewhere."""
+    faster_on_b200 = {
+        (8192, 3456): False, (8192, 1152): False, (8192, 4608): True,          # PixArt-Sigma
+        (2048, 6720): False, (2048, 2240): False, (2048, 5600): False,         # SANA
+        (4096, 1280): False, (4096, 10240): True,                              # SDXL
+        (17776, 9216): True, (17776, 3072): True, (17776, 12288): True,        # CogVideoX
+        (256, 1152): False,
+    }
+    for (M, N), pair in faster_on_b200.items():
+        assert tasq.tasq_gemm_choice(M, N, 148) is pair, (M, N)
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        M, N, sms = int(rng.integers(1, 40000)), int(rng.integers(1, 20000)), int(rng.integers(2, 200))
+        assert tasq.tasq_gemm_choice(M, N, sms) == tasq.tasq_gemm_choice(M, N, sms)
+    for bad in ((0, 8, 148), (8, 0, 148), (8, 8, 1)):
+        with pytest.raises(tasq.TasqError) as ei:
+            tasq.tasq_gemm_choice(*bad)
+        assert ei.value.status == tasq.TASQ_ERR_INVALID_ARG

@@ -73,6 +73,7 @@ def _load():
         "tasq_debug_gemm": [P, P, P, i64, i32, i32, P, i64, i32, P],
         "tasq_debug_stuck_wait": [P, P],
         "tasq_debug_set_gemm_mode": [P, i32],
+        "tasq_gemm_choice": [i64, i32, i32, ctypes.POINTER(i32)],
         "tasq_debug_set_mask_mode": [P, i32],
         "tasq_get_schedule": [P, P, P],
         "tasq_linear_forward_group": [P, P, i64, i64, P, i32, i32, P, P, P],
@@ -245,6 +246,13 @@ def tasq_debug_gemm(ctx: Context, xq, s_x, M: int, layer: int, step: int, y, ldy
 
 def tasq_debug_set_gemm_mode(ctx: Context, mode: int) -> None:
     _check(lib.tasq_debug_set_gemm_mode(ctx, int(mode)))
+
+
+def tasq_gemm_choice(M: int, N: int, num_sms: int) -> bool:
+    """True when the automatic choice runs this GEMM on CTA pairs; host-only, needs no device."""
+    pair = ctypes.c_int32(0)
+    _check(lib.tasq_gemm_choice(int(M), int(N), int(num_sms), ctypes.byref(pair)))
+    return bool(pair.value)
 
 
 def tasq_debug_set_prologue_mode(ctx: Context, mode: int) -> None:

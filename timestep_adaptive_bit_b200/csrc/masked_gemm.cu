@@ -10,7 +10,7 @@
 // de Hardware"). The bit width is read from the device schedule table inside the kernel, so a
 // new step needs no new weights and no different kernel.
 //
-// Design (one persistent CTA per SM, warp-specialised, 448 threads; the pair kernel in
+// Design (one persistent CTA per SM, warp-specialised, 576 threads; the pair kernel in
 // masked_gemm_pair.cu shares the roles and the epilogue):
 //   tile            128 output channels x 256 tokens; the weight tile is the MMA's A operand
 //                   (M = 128), the activation-code tile its B operand (N = 256); K advances in

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 #include <cstdio>
@@ -271,27 +272,39 @@ tasq_status run_prologue(tasq_ctx* c, int32_t layer, int32_t step, const std::ve
   return TASQ_OK;
 }
 
-// Which GEMM kernel finishes first. Both are persistent, so time = waves of tiles x time per
-// tile. Measured on B200: at the same wave count the CTA pair (256 x 256 tiles) beats one CTA
-// per 128 x 256 tile only once each CTA runs a long mainloop (1.14x at 12 waves x 24 K blocks,
-// CogVideoX proj). With a few hundred K blocks or less per CTA it loses up to 5 % (cluster
-// set-up and the pair's exit handshake), and with more waves it loses outright.
-bool prefer_pair(int64_t M, int64_t N, int64_t num_kb, int num_sms) {
-  const int64_t t1 = ((M + 255) / 256) * ((N + 127) / 128);
-  const int64_t t2 = ((M + 255) / 256) * ((N + 255) / 256);
+}  // namespace
+
+namespace tasq {
+
+// Which GEMM kernel finishes first. Both kernels are persistent, so a launch takes (waves of
+// tiles) x (time per tile). CUDA-event timings of single launches on B200, over both kernels on
+// the PixArt-Sigma, SANA, SDXL and CogVideoX shapes, fixed the rule:
+//   * with fewer waves the CTA pair (256 x 256 tiles) wins outright, with more it loses;
+//   * with equal waves the pair wins from four waves up (6 % on PixArt-Sigma fc1 and SDXL ff1,
+//     3-9 % on CogVideoX) and loses up to 9 % at one or two waves (SANA proj and fc2), where its
+//     cluster set-up and exit handshake are not amortised; at three it is level or behind.
+// Narrower token tiles (64 .. 224 tokens, both kernels) were measured as well: a tile's time
+// shrinks much less than its width, so they lost everywhere but on a few wave-quantised shapes,
+// and won there by 3 % at most.
+bool gemm_use_pair(int64_t M, int64_t N, int num_sms) {
+  const int64_t m_tiles = (M + kGemmTileTok - 1) / kGemmTileTok;
+  const int64_t t1 = m_tiles * ((N + kGemmTileCh - 1) / kGemmTileCh);
+  const int64_t t2 = m_tiles * ((N + kGemmPairTile - 1) / kGemmPairTile);
   const int64_t slots1 = num_sms, slots2 = num_sms / 2;
   const int64_t w1 = (t1 + slots1 - 1) / slots1;
   const int64_t w2 = (t2 + slots2 - 1) / slots2;
-  if (w2 < w1) return true;
-  return w2 == w1 && w1 * num_kb >= 200;
+  return w2 < w1 || (w2 == w1 && w1 >= 4);
 }
+
+}  // namespace tasq
+
+namespace {
 
 // GEMM of (layer, step). premasked: the weights come masked from masked-weight slot `slot`.
 tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq, const float* sx, int64_t M,
                      void* y, int64_t ldy, tasq::OutKind out, bool premasked, cudaStream_t s, int32_t slot = 0) {
   const LayerInfo& L = c->layers[layer];
-  const int64_t num_kb = (L.Kp + tasq::kGemmBlockK - 1) / tasq::kGemmBlockK;
-  const bool pair = c->gemm_mode == 2 || (c->gemm_mode == 0 && prefer_pair(M, L.N, num_kb, c->num_sms));
+  const bool pair = c->gemm_mode == 2 || (c->gemm_mode == 0 && tasq::gemm_use_pair(M, L.N, c->num_sms));
   const int tile_tok = pair ? tasq::kGemmPairTile : tasq::kGemmTileTok;
   const int tile_ch = pair ? tasq::kGemmPairTile : tasq::kGemmTileCh;
   CUtensorMap tx;
@@ -732,6 +745,14 @@ tasq_status tasq_debug_set_gemm_mode(tasq_ctx* c, int32_t mode) {
   if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
   if (mode < 0 || mode > 2) return fail(TASQ_ERR_INVALID_ARG, "mode must be 0, 1 or 2");
   c->gemm_mode = mode;
+  return TASQ_OK;
+}
+
+tasq_status tasq_gemm_choice(int64_t M, int32_t N, int32_t num_sms, int32_t* pair) {
+  g_last_error.clear();
+  if (pair == nullptr) return fail(TASQ_ERR_INVALID_ARG, "pair is NULL");
+  if (M <= 0 || N <= 0 || num_sms <= 1) return fail(TASQ_ERR_INVALID_ARG, "M and N must be positive, num_sms > 1");
+  *pair = tasq::gemm_use_pair(M, N, num_sms) ? 1 : 0;
   return TASQ_OK;
 }
 

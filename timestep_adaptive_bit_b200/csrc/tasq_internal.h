@@ -107,6 +107,10 @@ constexpr int kGemmTileTok = 256;   // activation rows per tile
 constexpr int kGemmBlockK = 128;    // K bytes per pipeline stage
 constexpr int kGemmStoreBox = 32;   // outputs leave in 32 x 32 TMA store boxes
 
+// Whether the automatic choice runs a GEMM of M tokens and N channels on CTA pairs rather than
+// one CTA per tile (defined in tasq_api.cu, with the measurements behind it).
+bool gemm_use_pair(int64_t M, int64_t N, int num_sms);
+
 cudaError_t launch_stuck_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t stream);
 
 // Whether kernels are launched with programmatic dependent launch, so that a kernel's setup
