@@ -328,6 +328,42 @@ def run_step(T, ctx, wl, xs, ys, step, stream):
                                             [ys[n] for n in Ns], Ns, stream)
 
 
+def time_same_traffic_copies(torch, wl, xs, stream, steps: int = 5):
+    """The prologue's yardstick at its own sizes: for every prologue launch of a step, one
+    device-to-device copy that moves the same DRAM traffic (half read from that launch's input
+    tensor, half written), each bracketed by CUDA events the way the per-kernel trace brackets a
+    prologue. Returns the copies' GB/s: summed traffic over summed event time."""
+    M = wl.tokens
+    per = len(wl.block_layers)
+    plan = wl.forward_plan()
+    sizes = {}
+    for group in plan:
+        K = wl.block_layers[group[0]][1]
+        traffic = 2 * M * K + M * wl.kp(K) + 4 * M
+        sizes[group[0]] = (traffic, (traffic // 2) // 16 * 16)
+    dst = torch.empty((max(nb for _, nb in sizes.values()),), dtype=torch.uint8, device=xs[0].device)
+    pairs = []
+    with torch.cuda.stream(stream):
+        for rep in range(steps + 1):
+            for b in range(wl.blocks):
+                for group in plan:
+                    traffic, nb = sizes[group[0]]
+                    src = xs[b * per + group[0]].view(torch.uint8).reshape(-1)[:nb]
+                    if rep == 0:   # warm-up pass
+                        dst[:nb].copy_(src, non_blocking=True)
+                        continue
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    dst[:nb].copy_(src, non_blocking=True)
+                    e1.record(stream)
+                    pairs.append((traffic, e0, e1))
+    torch.cuda.synchronize()
+    total_bytes = sum(t for t, _, _ in pairs)
+    total_ms = sum(e0.elapsed_time(e1) for _, e0, e1 in pairs)
+    return total_bytes / (total_ms / 1e3) / 1e9 if total_ms > 0 else None
+
+
 def launches_per_step(wl) -> int:
     """Kernels one step launches: a prologue per input, a GEMM per linear."""
     return wl.blocks * (len(wl.forward_plan()) + len(wl.block_layers))
@@ -561,6 +597,7 @@ def main(argv=None):
 
     # ---- next row: the on-device DMPQ predictor on the block's first input and last output
     dmpq = time_dmpq(T, torch, ctx, wl, xs, ys, stream)
+    copy_gbs = time_same_traffic_copies(torch, wl, xs, stream)
 
     peaks, peak_kind = load_peaks()
     int8_burst = peaks["bf16_tflops"] * INT8_OVER_BF16
@@ -606,7 +643,9 @@ def main(argv=None):
                      "frac_of_sustained": (gemm_tops / int8_sust) if gemm_tops else None},
         "prologue_roofline": {"bound": "hbm", "achieved": pro_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                               "frac": (pro_gbs / peaks["hbm_gbs"]) if pro_gbs else None,
-                              "frac_of_8000": (pro_gbs / 8000.0) if pro_gbs else None},
+                              "frac_of_8000": (pro_gbs / 8000.0) if pro_gbs else None,
+                              "same_traffic_copy_gbs": copy_gbs,
+                              "frac_of_same_traffic_copy": (pro_gbs / copy_gbs) if (pro_gbs and copy_gbs) else None},
         "gemm_share_of_step": trace["gemm_ms"] / max(traced_ms, 1e-9) if trace["gemm_ms"] else None,
         "kernel_timing": f"per-kernel CUDA events in a separate pass of {trace_steps} steps "
                          f"({traced_ms / trace_steps:.3f} ms per step with the events); the timed steps run "
