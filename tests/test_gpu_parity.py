@@ -98,6 +98,33 @@ def test_prologue_matches_oracle(T, n, K, M, pmode):
     assert T.tasq_get_device_status(ctx) == 0
 
 
+# rows whose transform is exact and whose scaled values are exact ties: z = blockwise x H_n holds
+# 254 once and small odd integers elsewhere, so a = 254, fp32(127 / a) = 0.5 and every other
+# z * 0.5 is a half-integer. x = z H_n / n is a multiple of 1/n below 2^11 / n, exact in FP16, and
+# every butterfly sum of it is exact in FP32, so both sides see the same exact ties.
+@pytest.mark.parametrize("pmode", [1, 2])
+@pytest.mark.parametrize("n,blocks,M", [(64, 3, 37), (128, 2, 20), (64, 18, 600)])
+def test_prologue_exact_ties_round_to_even(T, n, blocks, M, pmode):
+    rng = np.random.default_rng(n * 1000 + blocks * 10 + M)
+    K = n * blocks
+    z = (2 * rng.integers(-3, 4, size=(M, K)) + 1).astype(np.float64)   # odd, |z| <= 7
+    z[np.arange(M), rng.integers(0, K, size=M)] = 254.0
+    H = oracle.sylvester_hadamard(n).astype(np.float64)
+    x = np.concatenate([z[:, b * n:(b + 1) * n] @ H / n for b in range(blocks)], axis=1)
+    assert np.array_equal(x.astype(np.float16).astype(np.float64), x)
+    x = x.astype(np.float16)
+    ctx = _ctx(T, [(64, K, np.zeros((64, K), np.int8), np.ones(64, np.float32))], 1, n, M)
+    T.tasq_debug_set_prologue_mode(ctx, pmode)
+    xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    sx = torch.empty((M,), dtype=torch.float32, device="cuda")
+    T.tasq_debug_quantize(ctx, _dev(x), M, K, 0, xq, sx, _stream())
+    torch.cuda.synchronize()
+    q_ref, sx_ref, _ = oracle.prologue(x, n)
+    assert np.array_equal(q_ref, np.rint(z / 2.0).astype(np.int8)), "oracle: ties to even"
+    assert np.array_equal(xq.cpu().numpy(), q_ref), "ties must round to even on the GPU too"
+    assert np.all(np.abs(sx.cpu().numpy().astype(np.float64) - sx_ref) <= 1e-6 * sx_ref)
+
+
 # ----------------------------------------------------------------------------- GEMM, exact
 # (GEMM kernel, mask placement): kernel 1 = one CTA per 128 x 256 tile, 2 = CTA pairs on
 # 256 x 256 tiles; placement 1 = every weight tile masked in shared memory inside the GEMM,
