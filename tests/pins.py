@@ -239,3 +239,120 @@ def check_dmpq(gamma_fn, bits_fn, sums_fn):
     big = np.full(1 << 22, 65504, dtype=np.float16)
     num, den = sums_fn(big, -big)
     assert den == 65504 * (1 << 24) * (1 << 22) and num == 2 * den
+
+
+# ------------------------------------------------------------------------ NVFP4 branch
+def check_e2m1(encode, decode):
+    for row in _golden_rows("nvfp4_e2m1_examples.txt"):
+        v, c = (p.strip() for p in row.split("|"))
+        got = int(encode(np.array([float(v)]))[0])
+        assert got == int(c), f"E2M1 code of {v}: {got}, expected {c}"
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    # every code decodes to its grid value and encodes back to itself
+    for c in range(16):
+        val = float(decode(np.array([c]))[0])
+        mag = grid[c & 7]
+        assert val == (-mag if c & 8 else mag), f"E2M1 decode of {c}"
+        assert int(encode(np.array([val]))[0]) == (c if mag != 0 or c == 0 else 8), f"E2M1 round trip of {c}"
+    # brute force on a fine grid: nearest grid value, a tie to the even code, saturation at 6
+    t = np.arange(-8 * 64, 8 * 64 + 1) / 64.0
+    codes = encode(t).astype(np.int64)
+    for x, c in zip(t, codes):
+        d = np.abs(grid - min(abs(x), 6.0))
+        near = np.flatnonzero(d == d.min())
+        want = near[0] if len(near) == 1 else near[near % 2 == 0][0]
+        assert (c & 7) == want, f"E2M1 rounding of {x}"
+        assert (c >> 3) == (1 if x < 0 else 0), f"E2M1 sign of {x}"
+
+
+def check_e4m3(encode, decode):
+    import torch
+    for row in _golden_rows("nvfp4_e4m3_examples.txt"):
+        v, c = (p.strip() for p in row.split("|"))
+        got = int(encode(np.array([float(v)]))[0])
+        assert got == int(c, 16), f"E4M3 code of {v}: {got:#x}, expected 0x{c}"
+    codes = np.arange(127)
+    vals = decode(codes)
+    assert np.all(np.diff(vals) > 0), "E4M3 values must rise with the code"
+    assert np.array_equal(encode(vals).astype(np.int64), codes), "E4M3 round trip"
+    # an independent reference: PyTorch's float8_e4m3fn cast (round to nearest even) on the
+    # finite range, and on the decoded values themselves
+    ref_vals = torch.arange(0, 127, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(vals, ref_vals), "E4M3 values differ from PyTorch's float8_e4m3fn"
+    rng = np.random.default_rng(17)
+    s = np.concatenate([rng.uniform(0, 448, 4000), 2.0 ** rng.uniform(-12, 8.8, 4000), (vals[1:] + vals[:-1]) / 2])
+    s = np.minimum(s, 448.0).astype(np.float32).astype(np.float64)
+    ref = torch.from_numpy(s.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(encode(s).astype(np.uint8), ref), "E4M3 rounding differs from PyTorch's cast"
+    assert int(encode(np.array([1e6]))[0]) == 0x7E, "E4M3 must saturate at 448"
+
+
+def check_nvfp4_quantizer(quantize):
+    for row in _golden_rows("nvfp4_quant_examples.txt"):
+        z_s, c_s, s_s, sx_s = (p.strip() for p in row.split("|"))
+        z = np.array([[float(v) for v in z_s.split()]], dtype=np.float32)
+        codes, sb, s_x = quantize(z, 64)
+        assert np.array_equal(codes[0].astype(np.int64), [int(v) for v in c_s.split()]), f"NVFP4 codes of {z_s[:40]}"
+        assert np.array_equal(sb[0].astype(np.int64), [int(v, 16) for v in s_s.split()]), "NVFP4 block scales"
+        assert s_x[0] == float(sx_s), "NVFP4 token scale"
+    import oracle
+    rng = np.random.default_rng(19)
+    z = (rng.standard_normal((40, 256)) * rng.uniform(0.01, 100, size=(40, 1))).astype(np.float32)
+    z[:, 32:48] *= 1e-3            # a quiet block
+    z[5] = 0.0
+    codes, sb, s_x = quantize(z, 64)
+    e = oracle.e2m1_decode(codes)
+    s = np.repeat(oracle.e4m3_decode(sb), 16, axis=1)
+    a = np.abs(z).max(1).astype(np.float64)
+    live = a > 0
+    assert not np.any(codes[5] & 7) and s_x[5] == 0.0, "zero row"
+    # reconstruction: u / sb within half the local E2M1 spacing (plus the scale's own rounding)
+    u = z.astype(np.float64) * (2688.0 / np.where(live, a, 1.0))[:, None]
+    t = np.divide(u, s, out=np.zeros_like(u), where=s > 0)
+    spacing = np.where(np.abs(t) < 2, 0.5, np.where(np.abs(t) < 4, 1.0, 2.0))
+    ok = np.abs(e - np.clip(t, -6, 6)) <= 0.5 * spacing + 1e-6
+    assert np.all(ok[live]), "codes further than half a step from u / sb"
+    # each block's largest |u| lands at the top of the E2M1 range (4 or 6: the scale rounds)
+    top = np.abs(e).reshape(40, 16, 16).max(2)
+    assert np.all(top[live][sb[live] > 0] >= 4.0), "block absmax does not use the top of the range"
+    # the token's absmax block gets the largest scale, 448 (E4M3 0x7E)
+    assert np.all(sb[live].max(1) == 0x7E)
+    assert np.allclose(s_x[live], a[live] / (2688 * 8.0), rtol=1e-15)
+    # sign symmetry (zeros keep their own sign)
+    cn, sbn, _ = quantize(-z, 64)
+    assert np.array_equal(sbn, sb) and np.array_equal(cn & 7, codes & 7), "NVFP4 quantizer is not symmetric"
+
+
+def check_nvfp4_weights(quantize_w):
+    for row in _golden_rows("nvfp4_weight_examples.txt"):
+        w_s, c_s, s_s = (p.strip() for p in row.split("|"))
+        w = np.array([[int(v) for v in w_s.split()]], dtype=np.int8)
+        codes, sb = quantize_w(w)
+        assert np.array_equal(codes[0].astype(np.int64), [int(v) for v in c_s.split()]), "NVFP4 weight codes"
+        assert int(sb[0, 0]) == int(s_s, 16), "NVFP4 weight block scale"
+
+
+def check_nvfp4_gemm(gemm):
+    from fractions import Fraction
+    import oracle
+    rng = np.random.default_rng(23)
+    for (M, N, K) in ((1, 1, 16), (2, 3, 32), (3, 2, 64)):
+        ca = rng.integers(0, 16, size=(M, K)).astype(np.uint8)
+        cw = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+        sa = rng.integers(0, 127, size=(M, K // 16)).astype(np.uint8)
+        sw = rng.integers(0, 127, size=(N, K // 16)).astype(np.uint8)
+        acc = gemm(ca, sa, cw, sw)
+
+        def val_e2m1(c):
+            mag = [Fraction(0), Fraction(1, 2), Fraction(1), Fraction(3, 2), Fraction(2), Fraction(3), Fraction(4), Fraction(6)][c & 7]
+            return -mag if c & 8 else mag
+
+        def val_e4m3(c):
+            e, m = c >> 3, c & 7
+            return Fraction(m, 8) * Fraction(1, 64) if e == 0 else (1 + Fraction(m, 8)) * Fraction(2) ** (e - 7)
+
+        for i in range(M):
+            for j in range(N):
+                exact = sum(val_e2m1(int(ca[i, k])) * val_e4m3(int(sa[i, k // 16])) *
+                            val_e2m1(int(cw[j, k])) * val_e4m3(int(sw[j, k // 16])) for k in range(K))
+                assert Fraction(float(acc[i, j])) == exact, f"NVFP4 GEMM ({i}, {j}) != exact sum"

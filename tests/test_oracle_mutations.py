@@ -283,3 +283,57 @@ def test_mutation_dmpq_gamma(gamma_fn):
 @pytest.mark.parametrize("bits_fn", [_bits_ge, _bits_zero_stable])
 def test_mutation_dmpq_decision(bits_fn):
     _fails(pins.check_dmpq, oracle.dmpq_gamma, bits_fn, oracle.dmpq_l1_sums)
+
+
+# ---------------------------------------------------------------- NVFP4 branch
+def _e2m1_ties_away(t):
+    # ties away from zero instead of to the even mantissa
+    t = np.asarray(t, dtype=np.float64)
+    grid = oracle.E2M1_VALUES
+    mag = np.minimum(np.abs(t), 6.0)
+    best = np.array([int(np.flatnonzero(np.abs(grid - v) == np.abs(grid - v).min())[-1]) for v in mag.ravel()])
+    best = best.reshape(mag.shape)
+    return ((np.signbit(t).astype(np.int64) << 3) | best).astype(np.uint8)
+
+
+def _e4m3_truncating(s):
+    # rounds toward zero instead of to nearest
+    s = np.minimum(np.asarray(s, dtype=np.float64), 448.0)
+    v = oracle.E4M3_VALUES
+    return np.array([int(np.flatnonzero(v <= x)[-1]) for x in s.ravel()], dtype=np.uint8).reshape(s.shape)
+
+
+def _quant_range_4(z32, n):
+    # block scale b / 4 instead of b / 6: the block absmax no longer maps to the top code
+    import oracle.nvfp4_oracle as O
+    z32 = np.asarray(z32, dtype=np.float32)
+    a = np.abs(z32).max(1)
+    g = np.where(a > 0, np.float32(2688) / np.where(a > 0, a, 1), 0).astype(np.float32)
+    u = z32 * g[:, None]
+    blk = u.reshape(u.shape[0], -1, 16)
+    b = np.abs(blk).max(2)
+    sbc = oracle.e4m3_encode((b / np.float32(4)).astype(np.float32).astype(np.float64))
+    sb = oracle.e4m3_decode(sbc).astype(np.float32)
+    r = np.where(sb > 0, np.float32(1) / np.where(sb > 0, sb, 1), 0).astype(np.float32)
+    codes = oracle.e2m1_encode((blk * r[:, :, None]).astype(np.float64)).reshape(u.shape)
+    return codes, sbc, a.astype(np.float64) / (O.ACT_RANGE * math.sqrt(n))
+
+
+def _gemm_without_weight_scales(ca, sa, cw, sw):
+    return oracle.nvfp4_gemm(ca, sa, cw, np.full_like(sw, 0x38))   # every weight scale 1.0
+
+
+def test_mutation_e2m1_ties_away():
+    _fails(pins.check_e2m1, _e2m1_ties_away, oracle.e2m1_decode)
+
+
+def test_mutation_e4m3_truncation():
+    _fails(pins.check_e4m3, _e4m3_truncating, oracle.e4m3_decode)
+
+
+def test_mutation_nvfp4_scale_range():
+    _fails(pins.check_nvfp4_quantizer, _quant_range_4)
+
+
+def test_mutation_nvfp4_gemm_drops_weight_scales():
+    _fails(pins.check_nvfp4_gemm, _gemm_without_weight_scales)

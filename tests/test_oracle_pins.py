@@ -1,4 +1,6 @@
 """The oracle against what the pages and the mathematics fix (CPU only)."""
+import math
+
 import numpy as np
 import pytest
 
@@ -90,3 +92,39 @@ def test_outputs_fit_fp16(name):
 
 def test_dmpq_predictor():
     pins.check_dmpq(oracle.dmpq_gamma, oracle.dmpq_bits, oracle.dmpq_l1_sums)
+
+
+def test_nvfp4_e2m1():
+    pins.check_e2m1(oracle.e2m1_encode, oracle.e2m1_decode)
+
+
+def test_nvfp4_e4m3():
+    pins.check_e4m3(oracle.e4m3_encode, oracle.e4m3_decode)
+
+
+def test_nvfp4_quantizer():
+    pins.check_nvfp4_quantizer(oracle.nvfp4_quantize_activations)
+
+
+def test_nvfp4_weights():
+    pins.check_nvfp4_weights(oracle.nvfp4_quantize_weights)
+
+
+def test_nvfp4_gemm():
+    pins.check_nvfp4_gemm(oracle.nvfp4_gemm)
+
+
+def test_nvfp4_linear_approximates_the_real_product():
+    """End-to-end algebra: with the stored weights in the rotated basis (R3), y ~= x W_real^T,
+    W_real = s_w * W H_blk / sqrt(n), within the NVFP4 quantization error (a sanity check)."""
+    rng = np.random.default_rng(29)
+    M, N, K, n = 8, 12, 128, 64
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    w = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    s_w = rng.uniform(0.001, 0.01, size=N)
+    r = oracle.nvfp4_linear(x, w, s_w, n)
+    H = oracle.sylvester_hadamard(n).astype(np.float64)
+    Hb = np.kron(np.eye(K // n), H)
+    y_real = x.astype(np.float64) @ (w.astype(np.float64) * s_w[:, None] @ Hb / math.sqrt(n)).T
+    rel = np.linalg.norm(r["y"] - y_real) / np.linalg.norm(y_real)
+    assert rel < 0.2, f"NVFP4 W4A4 relative error {rel}"
