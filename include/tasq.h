@@ -101,7 +101,8 @@ tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, in
 
 /*
  * Replace the schedule table with bits_host [num_layers * num_steps] (host, row-major by layer,
- * every entry in [1, 8]; bits = 8 keeps all bit planes, bits = b keeps the top b planes).
+ * every entry in [0, 8]; bits = 8 keeps all bit planes, bits = b keeps the top b planes, and
+ * TASQ_NVFP4 (0) selects the NVFP4 step described below tasq_dmpq_update).
  * Stream-ordered: forwards enqueued on `stream` after this call see the new table. The host
  * array may be reused as soon as the call returns. No kernel is launched and the weight
  * buffer is never touched: the table is the only thing that changes between steps.
@@ -220,6 +221,48 @@ tasq_status tasq_dmpq_update(tasq_ctx* ctx, const void* block_in, int64_t ld_in,
                              int64_t ld_out, int64_t M, int32_t D, const int32_t* layers,
                              int32_t num_block_layers, int32_t step, double tau, int32_t bits_unstable,
                              int32_t bits_stable, double* gamma_out, void* stream);
+
+/*
+ * NVFP4 steps (6Bit-Diffusion, technical summary section 2.A: stable layers compressed to NVFP4,
+ * Blackwell's native 4-bit format, unstable ones kept in INT8). A schedule entry of TASQ_NVFP4
+ * (0) makes that (layer, step) an NVFP4 step: the forward's prologue launch quantizes the
+ * block-Hadamard activations to E2M1 codes with one UE4M3 scale per 16 elements along K and a
+ * per-token FP32 scale, and converts the layer's shared INT8 weights the same way (per output
+ * channel, s_w unchanged); a block-scaled tcgen05 GEMM (kind::mxf4nvf4) with FP32 accumulation
+ * and the same dequantizing epilogue follows. Entries 1..8 keep the INT8 path with that many
+ * weight bits. NVFP4 codes are packed two per byte along K, the lower-indexed element in the low
+ * nibble; block scales use 512-byte chunks, one per 128 rows x 64 elements of K, in which row r
+ * and 16-block j sit at byte (r % 32) * 16 + ((r % 128) / 32) * 4 + j, the chunks of a 128-row
+ * group in K order; K is padded with zero scales to a multiple of 256.
+ * tasq_linear_forward_noalloc and tasq_dmpq_update stay INT8-only.
+ */
+#define TASQ_NVFP4 0
+#define TASQ_NVFP4_RAW_ACC 2   /* out_kind of tasq_debug_gemm_nvfp4: raw FP32 accumulators */
+
+/* Host-only: bytes of the NVFP4 block scales of `rows` rows with Kp in-features (a multiple of 64). */
+tasq_status tasq_nvfp4_scale_bytes(int64_t rows, int32_t Kp, int64_t* bytes);
+
+/*
+ * Test hook: the NVFP4 prologue alone. x FP16 [M, K] (row stride ldx), codes [M, Kp / 2] bytes,
+ * scales tasq_nvfp4_scale_bytes(M, Kp) bytes (both 16-byte aligned, caller-owned device memory),
+ * s_x [M] FP32. Scales of padding rows and of K past Kp are left as they were.
+ */
+tasq_status tasq_debug_quantize_nvfp4(tasq_ctx* ctx, const void* x, int64_t M, int64_t ldx, int32_t layer,
+                                      void* codes, void* scales, float* s_x, void* stream);
+
+/* Test hook: the NVFP4 conversion of a layer's shared INT8 weights into codes [N, Kp / 2] and
+ * scales (tasq_nvfp4_scale_bytes(N, Kp) bytes), the K padding written as zero scales. */
+tasq_status tasq_debug_nvfp4_weights(tasq_ctx* ctx, int32_t layer, void* codes, void* scales, void* stream);
+
+/*
+ * Test hook: the NVFP4 GEMM on given activation codes, scales (as tasq_debug_quantize_nvfp4 writes
+ * them, with zero or finite scales wherever the layout has no row or no K) and s_x, against the
+ * layer's converted weights. out_kind TASQ_OUT_F16 / TASQ_OUT_BF16 write y = acc * s_x * s_w;
+ * TASQ_NVFP4_RAW_ACC writes the FP32 accumulators acc themselves (y float32 [M, ldy], ldy a
+ * multiple of 4).
+ */
+tasq_status tasq_debug_gemm_nvfp4(tasq_ctx* ctx, const void* codes, const void* scales, const float* s_x, int64_t M,
+                                  int32_t layer, void* y, int64_t ldy, int32_t out_kind, void* stream);
 
 /*
  * Test hook: which GEMM kernel later forwards of this context use. 0 (default) lets the library

@@ -465,7 +465,7 @@ def test_argument_errors_on_device(T):
     assert err(T.tasq_linear_forward, ctx, x, M, K, 0, -1, y, N, s) == T.TASQ_ERR_INVALID_ARG
     assert err(T.tasq_linear_forward, ctx, x, M, K, 0, 0, y, N + 3, s) == T.TASQ_ERR_INVALID_ARG
     assert err(T.tasq_linear_forward, ctx, x, -1, K, 0, 0, y, N, s) == T.TASQ_ERR_INVALID_ARG
-    assert err(T.tasq_set_schedule, ctx, np.array([[8, 0]], np.uint8), s) == T.TASQ_ERR_INVALID_ARG
+    assert err(T.tasq_set_schedule, ctx, np.array([[8, 10]], np.uint8), s) == T.TASQ_ERR_INVALID_ARG
     assert err(T.tasq_set_schedule, ctx, np.array([[9, 8]], np.uint8), s) == T.TASQ_ERR_INVALID_ARG
     assert err(T.tasq_debug_set_gemm_mode, ctx, 3) == T.TASQ_ERR_INVALID_ARG
     assert err(T.tasq_debug_set_mask_mode, ctx, 3) == T.TASQ_ERR_INVALID_ARG

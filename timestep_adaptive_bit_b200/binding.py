@@ -26,6 +26,8 @@ TASQ_ERR_TIMEOUT = 5
 
 TASQ_OUT_F16 = 0
 TASQ_OUT_BF16 = 1
+TASQ_NVFP4 = 0            # schedule entry of an NVFP4 step
+TASQ_NVFP4_RAW_ACC = 2    # tasq_debug_gemm_nvfp4: raw FP32 accumulators
 
 TASQ_DEVICE_TIMEOUT_PRODUCER = 0x1
 TASQ_DEVICE_TIMEOUT_MMA = 0x2
@@ -74,6 +76,10 @@ def _load():
         "tasq_debug_stuck_wait": [P, P],
         "tasq_debug_set_gemm_mode": [P, i32],
         "tasq_gemm_choice": [i64, i32, i32, ctypes.POINTER(i32)],
+        "tasq_nvfp4_scale_bytes": [i64, i32, ctypes.POINTER(i64)],
+        "tasq_debug_quantize_nvfp4": [P, P, i64, i64, i32, P, P, P, P],
+        "tasq_debug_nvfp4_weights": [P, i32, P, P, P],
+        "tasq_debug_gemm_nvfp4": [P, P, P, P, i64, i32, P, i64, i32, P],
         "tasq_debug_set_mask_mode": [P, i32],
         "tasq_get_schedule": [P, P, P],
         "tasq_linear_forward_group": [P, P, i64, i64, P, i32, i32, P, P, P],
@@ -231,6 +237,29 @@ def tasq_layer_info(ctx: Context, layer: int):
 
 def tasq_debug_quantize(ctx: Context, x, M: int, ldx: int, layer: int, xq, s_x, stream=None) -> None:
     _check(lib.tasq_debug_quantize(ctx, _ptr(x), int(M), int(ldx), int(layer), _ptr(xq), _ptr(s_x), _stream(stream)))
+
+
+def tasq_nvfp4_scale_bytes(rows: int, Kp: int) -> int:
+    """Bytes of the NVFP4 block scales of `rows` rows with Kp in-features (host-only)."""
+    out = ctypes.c_int64(0)
+    _check(lib.tasq_nvfp4_scale_bytes(int(rows), int(Kp), ctypes.byref(out)))
+    return int(out.value)
+
+
+def tasq_debug_quantize_nvfp4(ctx: Context, x, M: int, ldx: int, layer: int, codes, scales, s_x,
+                              stream=None) -> None:
+    _check(lib.tasq_debug_quantize_nvfp4(ctx, _ptr(x), int(M), int(ldx), int(layer), _ptr(codes), _ptr(scales),
+                                         _ptr(s_x), _stream(stream)))
+
+
+def tasq_debug_nvfp4_weights(ctx: Context, layer: int, codes, scales, stream=None) -> None:
+    _check(lib.tasq_debug_nvfp4_weights(ctx, int(layer), _ptr(codes), _ptr(scales), _stream(stream)))
+
+
+def tasq_debug_gemm_nvfp4(ctx: Context, codes, scales, s_x, M: int, layer: int, y, ldy: int, out_kind: int,
+                          stream=None) -> None:
+    _check(lib.tasq_debug_gemm_nvfp4(ctx, _ptr(codes), _ptr(scales), _ptr(s_x), int(M), int(layer), _ptr(y),
+                                     int(ldy), int(out_kind), _stream(stream)))
 
 
 def tasq_debug_gemm_s32(ctx: Context, xq, M: int, layer: int, step: int, acc, ld_acc: int, stream=None) -> None:

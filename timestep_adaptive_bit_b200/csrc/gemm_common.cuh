@@ -50,11 +50,13 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
 }
 
 // Two adjacent tokens of one channel: y = (acc * s_x) * s_w in FP32, then a packed FP16 / BF16
-// pair (first token in the low half).
-template <int OUT>
+// pair (first token in the low half). The accumulators are INT32 (the INT8 GEMM) or FP32 (the
+// block-scaled NVFP4 GEMM, ACC_F32).
+template <int OUT, bool ACC_F32 = false>
 __device__ __forceinline__ uint32_t out_pair(uint32_t a0, uint32_t a1, float2 sx, float sw) {
-  const float2 acc = make_float2(static_cast<float>(static_cast<int32_t>(a0)),
-                                 static_cast<float>(static_cast<int32_t>(a1)));
+  const float2 acc = ACC_F32 ? make_float2(__uint_as_float(a0), __uint_as_float(a1))
+                             : make_float2(static_cast<float>(static_cast<int32_t>(a0)),
+                                           static_cast<float>(static_cast<int32_t>(a1)));
   const float2 v = mul2(mul2(acc, sx), make_float2(sw, sw));
   if constexpr (OUT == static_cast<int>(OutKind::F16)) {
     const __half2 h = __floats2half2_rn(v.x, v.y);
@@ -75,12 +77,14 @@ __device__ __forceinline__ uint32_t out_pair(uint32_t a0, uint32_t a1, float2 sx
 //   stmatrix.trans writes token-major into the box, 16 bytes per row, through a 64-byte swizzle
 //   (chunk ^= (row >> 1) & 3) that keeps the eight rows of each matrix on distinct banks; the TMA
 //   store undoes the swizzle.
-//   INT32 (test hook): 32 x 32-bit TMEM loads, one value per lane per store, no swizzle.
+//   INT32 (test hook): 32 x 32-bit TMEM loads, one value per lane per store, no swizzle; the raw
+//   accumulator words (FP32 bits when ACC_F32).
+//   ACC_F32: the accumulators are FP32 (the NVFP4 GEMM) instead of INT32.
 //   ch_per_tile / ch_offset : output channels of tile nt start at nt * ch_per_tile + ch_offset.
 //   acc_full + 8 i          : local barrier the MMA side arrives on when accumulator i is ready.
 //   acc_empty + 8 i         : barrier (local, or in another CTA of the cluster when CLUSTER) that
 //                             each epilogue warp arrives on once, after reading accumulator i.
-template <int OUT, bool CLUSTER, int TOK>
+template <int OUT, bool CLUSTER, int TOK, bool ACC_F32 = false>
 __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorMap* tmap_y, uint32_t tmem_base,
                                               uint8_t* stage, float* sx_slice, int warp, int lane, int tile0,
                                               int tile_step, int num_tiles, int ch_per_tile, int ch_offset,
@@ -203,7 +207,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
 #pragma unroll
               for (int r = 0; r < 4; ++r) {
                 const int tl = 8 * r + 2 * (lane & 3);
-                const uint32_t pr = out_pair<OUT>(rr[4 * r + 2 * o], rr[4 * r + 2 * o + 1],
+                const uint32_t pr = out_pair<OUT, ACC_F32>(rr[4 * r + 2 * o], rr[4 * r + 2 * o + 1],
                                                   make_float2(sxc[tl], sxc[tl + 1]), sw[gg][o]);
                 if (ch < g.N) {
                   uint16_t* y = static_cast<uint16_t*>(g.y);
@@ -233,7 +237,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
           for (int o = 0; o < 2; ++o) {
             uint32_t p[4];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) p[r] = out_pair<OUT>(rr[4 * r + 2 * o], rr[4 * r + 2 * o + 1], sx2[r], sw[gg][o]);
+            for (int r = 0; r < 4; ++r) p[r] = out_pair<OUT, ACC_F32>(rr[4 * r + 2 * o], rr[4 * r + 2 * o + 1], sx2[r], sw[gg][o]);
             const uint32_t chunk = static_cast<uint32_t>(2 * gg + o);
             ptx::stmatrix_x4_trans(row_addr + 16u * (chunk ^ swz), p[0], p[1], p[2], p[3]);
           }

@@ -309,6 +309,186 @@ __global__ void __launch_bounds__(MAXT, MINB)
   if (seg == 0) a.s_x[row] = __fmul_rn(amax, a.sx_factor);
 }
 
+// ------------------------------------------------------------------------------ NVFP4 variant
+// The NVFP4 step of 6Bit-Diffusion (technical summary, section 2.A: the stable layers of a step
+// in NVFP4, Blackwell's 4-bit format, after the same block Hadamard). The thread layout, loads and
+// transform are those of the direct INT8 kernel; then per token u = z * fp32(2688 / a), and per
+// 16-block of a row b = max |u|, the UE4M3 scale sb = RNE(fp32(b / 6)) and the E2M1 codes
+// RNE(fp32(u * fp32(1 / sb))), both saturating; a block whose scale is 0 gets zero codes. The
+// thread's 32 channels are two whole 16-blocks: the .x halves of its register pairs and the .y
+// halves.
+
+// UE4M3 code of s >= 0, round to nearest even, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3_code(float s) {
+  uint16_t h;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(s), "f"(s));
+  return h & 0xFFu;
+}
+
+// Value of a UE4M3 code, exact (every E4M3 value is an FP16 value). The code sits in both bytes,
+// so either half of the FP16 pair holds it.
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  uint32_t h2;
+  const uint16_t both = static_cast<uint16_t>(code | (code << 8));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(both));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+
+// E2M1 codes of eight values (round to nearest even, saturating at 6), t[0] in the lowest nibble.
+__device__ __forceinline__ uint32_t e2m1_x8(const float (&t)[8]) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+      : "=r"(r)
+      : "f"(t[0]), "f"(t[1]), "f"(t[2]), "f"(t[3]), "f"(t[4]), "f"(t[5]), "f"(t[6]), "f"(t[7]));
+  return r;
+}
+
+__device__ __forceinline__ float2 mul2v(float2 a, float2 b) {
+  const uint64_t ua = *reinterpret_cast<const uint64_t*>(&a);
+  const uint64_t ub = *reinterpret_cast<const uint64_t*>(&b);
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(ua), "l"(ub));
+  return *reinterpret_cast<const float2*>(&r);
+}
+
+// Byte of row r, 16-block j in the chunked scale layout (see Nvfp4PrologueArgs).
+__device__ __forceinline__ int64_t nvfp4_sf_offset(int64_t r, int64_t j, int64_t chunks_per_group) {
+  return ((r >> 7) * chunks_per_group + (j >> 2)) * kNvfp4ChunkBytes + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (j & 3);
+}
+
+// NVFP4 codes and scale of the 16 INT8 weights w[0..15] (one block of one output channel).
+__device__ __forceinline__ void nvfp4_weight_block(const int8_t* w, uint8_t* codes, uint8_t* sf_byte) {
+  const uint4 q = *reinterpret_cast<const uint4*>(w);
+  const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+  float f[16];
+  int m = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int v = static_cast<int8_t>((words[i >> 2] >> (8 * (i & 3))) & 0xFFu);
+    f[i] = static_cast<float>(v);
+    m = max(m, abs(v));
+  }
+  const uint32_t sc = e4m3_code(__fdiv_rn(static_cast<float>(m), 6.0f));
+  const float d = e4m3_value(sc);
+  const float r = d > 0.0f ? __frcp_rn(d) : 0.0f;
+  float t0[8], t1[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    t0[i] = __fmul_rn(f[i], r);
+    t1[i] = __fmul_rn(f[8 + i], r);
+  }
+  uint2 out = make_uint2(e2m1_x8(t0), e2m1_x8(t1));
+  if (d == 0.0f) out = make_uint2(0u, 0u);
+  *reinterpret_cast<uint2*>(codes) = out;
+  *sf_byte = static_cast<uint8_t>(sc);
+}
+
+// Weight conversion of CTA `cta` of `num_ctas`: one thread per 16-block, then zero scales for
+// the blocks between Kp and Kp4, so that the GEMM's last stage multiplies zero codes by zero.
+__device__ __forceinline__ void nvfp4_weight_pass(const Nvfp4PrologueArgs& a, int64_t cta, int64_t num_ctas) {
+  // the previous GEMM may still read the converted weights: wait for it
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (cta == 0 && threadIdx.x == 0 && a.bits_table != nullptr && a.bits_table[a.bits_index] != 0)
+    atomicOr(a.status, TASQ_DEVICE_BAD_BITS);
+  const int64_t nb = a.Kp / kNvfp4Block;
+  const int64_t nb4 = nvfp4_kp4(a.Kp) / kNvfp4Block;
+  const int64_t chunks = nb4 / 4;
+  const int64_t stride = num_ctas * blockDim.x;
+  for (int64_t i = cta * blockDim.x + threadIdx.x; i < static_cast<int64_t>(a.N) * nb4; i += stride) {
+    const int64_t row = i / nb4, j = i - row * nb4;
+    uint8_t* sf = a.w_sf + nvfp4_sf_offset(row, j, chunks);
+    if (j < nb) nvfp4_weight_block(a.w + row * a.Kp + 16 * j, a.w_codes + row * (a.Kp / 2) + 8 * j, sf);
+    else *sf = 0;
+  }
+}
+
+template <int LANES, int MAXT, int MINB>
+__global__ void __launch_bounds__(MAXT, MINB)
+    prologue_nvfp4_kernel(const Nvfp4PrologueArgs a, const int rows_per_cta, const int row_ctas) {
+  if (static_cast<int>(blockIdx.x) >= row_ctas) {
+    nvfp4_weight_pass(a, blockIdx.x - row_ctas, gridDim.x - row_ctas);
+    return;
+  }
+  const int L = a.Kp >> 5;
+  const int tid = threadIdx.x;
+  const int r_local = tid / L;
+  const int seg = tid - r_local * L;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + r_local;
+  const bool active = r_local < rows_per_cta && row < a.M;
+
+  // x may be the previous kernel's output, and the previous GEMM may still read the codes
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  __shared__ unsigned int row_max[kMaxRowsPerCta];
+  if (tid < rows_per_cta) row_max[tid] = 0u;
+  __syncthreads();
+
+  const int c0 = seg * 32;
+  float2 v[16];
+  {
+    uint32_t u[16];
+    const __half* src = static_cast<const __half*>(a.x) + row * a.ldx + c0;
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+      uint32_t* ug = u + 8 * g;
+      const int e0 = c0 + 16 * g;
+      if (active && e0 + 16 <= a.K) {
+        const uint4 p0 = ld_16B(src + 16 * g), p1 = ld_16B(src + 16 * g + 8);
+        ug[0] = p0.x; ug[1] = p0.y; ug[2] = p0.z; ug[3] = p0.w;
+        ug[4] = p1.x; ug[5] = p1.y; ug[6] = p1.z; ug[7] = p1.w;
+      } else if (active && e0 + 8 <= a.K) {
+        const uint4 p0 = ld_16B(src + 16 * g);
+        ug[0] = p0.x; ug[1] = p0.y; ug[2] = p0.z; ug[3] = p0.w;
+        ug[4] = 0u; ug[5] = 0u; ug[6] = 0u; ug[7] = 0u;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ug[i] = 0u;
+      }
+    }
+    to_pairs(u, v);
+  }
+  fwht_segment<LANES>(v, seg, 1);
+  const float mx = absmax_segment(v);
+  if (active) atomicMax(&row_max[r_local], __float_as_uint(mx));
+  __syncthreads();
+  if (!active) return;
+  const float amax = __uint_as_float(row_max[r_local]);
+  const float g = amax > 0.0f ? __fdiv_rn(kNvfp4Range, amax) : 0.0f;
+  float b0 = 0.0f, b1 = 0.0f;
+#pragma unroll
+  for (int p = 0; p < 16; ++p) {
+    v[p] = mul2(v[p], g);
+    b0 = fmaxf(b0, fabsf(v[p].x));
+    b1 = fmaxf(b1, fabsf(v[p].y));
+  }
+  const uint32_t s0 = e4m3_code(__fdiv_rn(b0, 6.0f)), s1 = e4m3_code(__fdiv_rn(b1, 6.0f));
+  const float d0 = e4m3_value(s0), d1 = e4m3_value(s1);
+  const float2 r = make_float2(d0 > 0.0f ? __frcp_rn(d0) : 0.0f, d1 > 0.0f ? __frcp_rn(d1) : 0.0f);
+  float t0[8], t1[8], t2[8], t3[8];
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const float2 lo = mul2v(v[p], r), hi = mul2v(v[p + 8], r);
+    t0[p] = lo.x;   // block 0: channels c0 .. c0 + 7
+    t1[p] = hi.x;   //          c0 + 8 .. c0 + 15
+    t2[p] = lo.y;   // block 1: c0 + 16 .. c0 + 23
+    t3[p] = hi.y;   //          c0 + 24 .. c0 + 31
+  }
+  uint32_t w0 = e2m1_x8(t0), w1 = e2m1_x8(t1), w2 = e2m1_x8(t2), w3 = e2m1_x8(t3);
+  if (d0 == 0.0f) w0 = w1 = 0u;
+  if (d1 == 0.0f) w2 = w3 = 0u;
+  st_16B(a.codes + row * (a.Kp / 2) + c0 / 2, w0, w1, w2, w3);
+  const int64_t chunks = nvfp4_kp4(a.Kp) / 64;
+  *reinterpret_cast<uint16_t*>(a.sf + nvfp4_sf_offset(row, c0 >> 4, chunks)) = static_cast<uint16_t>(s0 | (s1 << 8));
+  if (seg == 0) a.s_x[row] = __fmul_rn(amax, a.sx_factor);
+}
+
 // ------------------------------------------------------------------------------ bulk-fed variant
 constexpr int kFedMaxCompute = 992;           // compute threads per CTA (one CTA per SM)
 constexpr int kFedMaxStageBytes = 50 * 1024;
@@ -601,6 +781,52 @@ bool try_launch_fed(const PrologueArgs& a, cudaStream_t stream, cudaError_t* err
 }
 
 }  // namespace
+
+cudaError_t launch_prologue_nvfp4(const Nvfp4PrologueArgs& a, cudaStream_t stream) {
+  const bool weights = a.w != nullptr;
+  if (a.M <= 0 && !weights) return cudaSuccess;
+  if (a.Kp % a.n != 0 || (a.n != 64 && a.n != 128) || a.K % 8 != 0) return cudaErrorInvalidValue;
+  if (a.M > 0 && (reinterpret_cast<uintptr_t>(a.x) % 16 != 0 || a.ldx % 8 != 0 ||
+                  reinterpret_cast<uintptr_t>(a.codes) % 16 != 0 || reinterpret_cast<uintptr_t>(a.sf) % 2 != 0))
+    return cudaErrorInvalidValue;
+  if (weights && (reinterpret_cast<uintptr_t>(a.w) % 16 != 0 || reinterpret_cast<uintptr_t>(a.w_codes) % 8 != 0 ||
+                  a.status == nullptr || a.N <= 0))
+    return cudaErrorInvalidValue;
+  const int L = a.Kp / 32;
+  if (L > kMaxThreads) return cudaErrorInvalidValue;
+  const bool small = L <= kSmallThreads;
+  int R = 1, threads = 256;
+  int64_t row_ctas = 0;
+  if (a.M > 0) {
+    R = pick_rows(L, small ? kSmallThreads : kMaxThreads);
+    threads = ((R * L + 31) / 32) * 32;
+    row_ctas = (a.M + R - 1) / R;
+  }
+  int64_t weight_ctas = 0;
+  if (weights) {
+    const int64_t blocks = static_cast<int64_t>(a.N) * (nvfp4_kp4(a.Kp) / kNvfp4Block);
+    weight_ctas = (blocks + threads - 1) / threads;
+    if (weight_ctas > kMaxWeightCtas) weight_ctas = kMaxWeightCtas;
+  }
+  const int64_t grid = row_ctas + weight_ctas;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = use_pdl() ? 1 : 0;
+  const int rc = static_cast<int>(row_ctas);
+  if (small) {
+    if (a.n == 64) return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<2, kSmallThreads, 4>, a, R, rc);
+    return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<4, kSmallThreads, 4>, a, R, rc);
+  }
+  if (a.n == 64) return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<2, kMaxThreads, 1>, a, R, rc);
+  return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<4, kMaxThreads, 1>, a, R, rc);
+}
 
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
   const bool weights = a.num_w > 0;

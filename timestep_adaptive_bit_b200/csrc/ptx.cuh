@@ -144,6 +144,27 @@ __device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// Block-scaled NVFP4 MMA, D (FP32, TMEM) (+)= A x B^T: A and B hold E2M1 codes (two per byte,
+// K-major) in shared memory, and every row of A and of B has one UE4M3 scale per 16 elements
+// along K, read from TMEM at sfa_tmem / sfb_tmem (kind::mxf4nvf4, scale_vec::4X: K = 64 per
+// instruction, four scales per row, one 32-bit TMEM word per row).
+__device__ __forceinline__ void mma_nvfp4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Copy a 512-byte block of shared memory, 32 rows of 16 bytes, into TMEM: row i goes to lane i of
+// each of the four 32-lane quarters, as four consecutive 32-bit columns starting at taddr.
+// Issued by one thread; it runs in order with the MMAs that thread issues.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 operation this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -251,6 +272,23 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(2u) << 61;
   return d;
+}
+
+// Descriptor of an unswizzled K-major block of 16-byte rows stored back to back: core matrices
+// of 8 rows x 16 bytes, 128 bytes apart along the rows (stride byte offset), one along K.
+__device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(128u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;   // layout type 0: no swizzle
+}
+
+// Instruction descriptor of tcgen05.mma kind::mxf4nvf4 with block scales: A and B E2M1 (format 1
+// in bits [7,10) and [10,13)), both K-major, UE4M3 scales (bit 23 = 0), N >> 3 in bits [17,23),
+// M >> 4 in bits [24,29), scale-factor byte ids 0, K = 64.
+__host__ __device__ constexpr uint32_t idesc_nvfp4(uint32_t M, uint32_t N) {
+  return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
 // Instruction descriptor of tcgen05.mma kind::i8: S32 accumulator (bits [4,6) = 2), A and B

@@ -132,13 +132,15 @@ struct tasq_ctx {
   int8_t* d_w = nullptr;
   float* d_sw = nullptr;
   uint8_t* d_bits = nullptr;
-  int8_t* d_xq = nullptr;
+  int8_t* d_xq = nullptr;               // INT8 codes [M, Kp], or NVFP4 codes [M, Kp / 2]
+  uint8_t* d_sf4 = nullptr;             // NVFP4 block scales of the activations (chunked layout)
   float* d_sx = nullptr;
   uint32_t* d_status = nullptr;
   uint64_t* d_dmpq = nullptr;          // per-CTA partial sums of the DMPQ predictor
   unsigned int* d_dmpq_arrived = nullptr;   // its CTA arrival counter (zero between calls)
   uint64_t wait_limit_ns = 1000000000ull;
   float sx_factor = 0.0f;
+  float sx_factor4 = 0.0f;              // NVFP4: fp32(1 / (2688 sqrt(n)))
   int32_t gemm_mode = 0;   // 0 automatic, 1 one CTA per tile, 2 CTA pairs
   int32_t mask_mode = 0;   // 0 automatic, 1 mask inside the GEMM, 2 mask ahead in the prologue launch
   int32_t prologue_mode = 0;   // 0 automatic, 1 direct-load prologue, 2 bulk-fed prologue where it fits
@@ -166,6 +168,7 @@ void free_ctx(tasq_ctx* c) {
   cudaFree(c->d_sw);
   cudaFree(c->d_bits);
   cudaFree(c->d_xq);
+  cudaFree(c->d_sf4);
   cudaFree(c->d_sx);
   cudaFree(c->d_status);
   cudaFree(c->d_dmpq);
@@ -269,6 +272,93 @@ tasq_status run_prologue(tasq_ctx* c, int32_t layer, int32_t step, const std::ve
     if (!g_last_error.empty()) return fail(TASQ_ERR_CUDA, "prologue launch: " + g_last_error);
     return fail_cuda(e, "prologue launch");
   }
+  return TASQ_OK;
+}
+
+// ---------------------------------------------------------------- NVFP4 step
+bool nvfp4_step(const tasq_ctx* c, int32_t layer, int32_t step) {
+  return c->bits_host[static_cast<size_t>(layer) * c->num_steps + step] == 0;
+}
+
+// The NVFP4 weights of a layer live in masked-weight slot `slot`: codes [N, Kp / 2] at its start,
+// block scales from the next 512-byte boundary.
+uint8_t* nvfp4_w_codes(const tasq_ctx* c, int32_t slot) { return reinterpret_cast<uint8_t*>(wk_slot(c, slot)); }
+uint8_t* nvfp4_w_sf(const tasq_ctx* c, int32_t layer, int32_t slot) {
+  const LayerInfo& L = c->layers[layer];
+  return nvfp4_w_codes(c, slot) + round_up(static_cast<size_t>(L.N) * L.Kp / 2, 512);
+}
+
+// NVFP4 prologue launch: activations (M > 0) into codes / sf / sx, and, when w_codes is set, the
+// layer's weights converted into w_codes / w_sf. step < 0: no schedule check.
+tasq_status run_prologue_nvfp4(tasq_ctx* c, int32_t layer, int32_t step, const void* x, int64_t M, int64_t ldx,
+                               uint8_t* codes, uint8_t* sf, float* sx, uint8_t* w_codes, uint8_t* w_sf,
+                               cudaStream_t s) {
+  const LayerInfo& L = c->layers[layer];
+  tasq::Nvfp4PrologueArgs a{};
+  a.x = x;
+  a.ldx = ldx;
+  a.K = L.K;
+  a.Kp = L.Kp;
+  a.n = c->n;
+  a.M = M;
+  a.codes = codes;
+  a.sf = sf;
+  a.s_x = sx;
+  a.sx_factor = c->sx_factor4;
+  if (w_codes != nullptr) {
+    a.w = c->d_w + L.w_off;
+    a.w_codes = w_codes;
+    a.w_sf = w_sf;
+    a.N = L.N;
+    a.bits_table = c->d_bits;
+    a.bits_index = layer * c->num_steps + (step < 0 ? 0 : step);
+    if (step < 0) a.bits_table = nullptr;
+  }
+  a.status = c->d_status;
+  cudaError_t e = tasq::launch_prologue_nvfp4(a, s);
+  if (e != cudaSuccess) return fail_cuda(e, "NVFP4 prologue launch");
+  return TASQ_OK;
+}
+
+// NVFP4 GEMM of (layer, step) on the given activation codes and the weights in slot `slot`.
+// step < 0: no schedule check. out S32 writes the raw FP32 accumulators.
+tasq_status run_gemm_nvfp4(tasq_ctx* c, int32_t layer, int32_t step, const uint8_t* codes, const uint8_t* sf,
+                           const float* sx, int64_t M, void* y, int64_t ldy, tasq::OutKind out, int32_t slot,
+                           cudaStream_t s) {
+  const LayerInfo& L = c->layers[layer];
+  const int64_t kp4 = tasq::nvfp4_kp4(L.Kp);
+  CUtensorMap tw, tx, ty;
+  tasq_status st = make_tmap_u8(&tw, nvfp4_w_codes(c, slot), static_cast<uint64_t>(L.Kp / 2),
+                                static_cast<uint64_t>(L.N), 128, 128);
+  if (st == TASQ_OK)
+    st = make_tmap_u8(&tx, codes, static_cast<uint64_t>(L.Kp / 2), static_cast<uint64_t>(M), 128, 128);
+  if (st != TASQ_OK) return st;
+  const CUtensorMapDataType dt = out == tasq::OutKind::S32    ? CU_TENSOR_MAP_DATA_TYPE_INT32
+                                 : out == tasq::OutKind::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  st = make_tmap_out(&ty, y, dt, out == tasq::OutKind::S32 ? 4u : 2u, static_cast<uint64_t>(L.N),
+                     static_cast<uint64_t>(M), static_cast<uint64_t>(ldy));
+  if (st != TASQ_OK) return st;
+  tasq::GemmArgs g{};
+  g.M = static_cast<int32_t>(M);
+  g.N = L.N;
+  g.num_kb = static_cast<int32_t>(kp4 / 256);
+  g.num_m_tiles = static_cast<int32_t>((M + 127) / 128);
+  g.num_n_tiles = (L.N + 127) / 128;
+  g.bits_table = step < 0 ? nullptr : c->d_bits;
+  g.bits_index = layer * c->num_steps + (step < 0 ? 0 : step);
+  g.s_x = sx;
+  g.s_w = c->d_sw + L.sw_off;
+  g.y = y;
+  g.ldy = ldy;
+  g.status = c->d_status;
+  g.wait_limit_ns = c->wait_limit_ns;
+  tasq::Nvfp4GemmArgs f{};
+  f.w_sf = nvfp4_w_sf(c, layer, slot);
+  f.x_sf = sf;
+  f.sf_chunks = static_cast<int32_t>(kp4 / 64);
+  cudaError_t e = tasq::launch_gemm_nvfp4(tw, tx, ty, g, f, out, c->num_sms, s);
+  if (e != cudaSuccess) return fail_cuda(e, "NVFP4 GEMM launch");
   return TASQ_OK;
 }
 
@@ -391,6 +481,10 @@ tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, in
     info[l] = LayerInfo{d.N, d.K, Kp, w_bytes, sw_count};
     w_bytes = round_up(w_bytes + static_cast<size_t>(d.N) * Kp, 1024);
     if (static_cast<size_t>(d.N) * Kp > wk_bytes) wk_bytes = static_cast<size_t>(d.N) * Kp;
+    // an NVFP4 step keeps the layer's converted weights in the same slot: codes, then scales
+    const size_t f4 = round_up(static_cast<size_t>(d.N) * Kp / 2, 512) +
+                      static_cast<size_t>(tasq::nvfp4_sf_bytes(d.N, Kp));
+    if (f4 > wk_bytes) wk_bytes = f4;
     sw_count = round_up(sw_count + d.N, 64);
     if (Kp > kp_max) kp_max = Kp;
   }
@@ -417,6 +511,7 @@ tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, in
   c->kp_max = kp_max;
   c->layers = info;
   c->sx_factor = static_cast<float>(1.0 / (127.0 * std::sqrt(static_cast<double>(hadamard_n))));
+  c->sx_factor4 = static_cast<float>(1.0 / (tasq::kNvfp4Range * std::sqrt(static_cast<double>(hadamard_n))));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   auto bail = [&](cudaError_t err, const char* what) {
@@ -436,6 +531,10 @@ tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, in
     return bail(e, "cudaMalloc(workspace codes)");
   if ((e = cudaMalloc(&c->d_sx, static_cast<size_t>(max_tokens) * sizeof(float))) != cudaSuccess)
     return bail(e, "cudaMalloc(workspace scales)");
+  const size_t sf4_bytes = static_cast<size_t>(tasq::nvfp4_sf_bytes(max_tokens, kp_max));
+  if ((e = cudaMalloc(&c->d_sf4, sf4_bytes)) != cudaSuccess) return bail(e, "cudaMalloc(NVFP4 block scales)");
+  // scales past a layer's Kp and rows past M are read by the NVFP4 GEMM: keep them finite
+  if ((e = cudaMemsetAsync(c->d_sf4, 0, sf4_bytes, s)) != cudaSuccess) return bail(e, "cudaMemsetAsync(NVFP4 scales)");
   if ((e = cudaMalloc(&c->d_status, sizeof(uint32_t))) != cudaSuccess) return bail(e, "cudaMalloc(status)");
   if ((e = cudaMalloc(&c->d_dmpq, 4 * sizeof(uint64_t) * static_cast<size_t>(c->num_sms) * tasq::kDmpqCtasPerSm)) !=
       cudaSuccess)
@@ -483,9 +582,9 @@ tasq_status tasq_set_schedule(tasq_ctx* c, const uint8_t* bits_host, void* strea
   if (st != TASQ_OK) return st;
   const size_t table = static_cast<size_t>(c->num_layers) * c->num_steps;
   for (size_t i = 0; i < table; ++i) {
-    if (bits_host[i] < 1 || bits_host[i] > 8)
+    if (bits_host[i] > 8)
       return fail(TASQ_ERR_INVALID_ARG, "bits[" + std::to_string(i) + "] = " + std::to_string(bits_host[i]) +
-                                            " outside [1, 8]");
+                                            " outside [0, 8] (0: NVFP4, 1..8: INT8 width)");
   }
   cudaError_t e = cudaMemcpyAsync(c->d_bits, bits_host, table, cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e, "copy of schedule");
@@ -509,13 +608,31 @@ tasq_status tasq_linear_forward(tasq_ctx* c, const void* x, int64_t M, int64_t l
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   TraceRec* tr = c->trace_count < c->trace_cap ? &c->trace[c->trace_count] : nullptr;
+  const tasq::OutKind out = c->out_dtype == TASQ_OUT_BF16 ? tasq::OutKind::BF16 : tasq::OutKind::F16;
+  if (nvfp4_step(c, layer, step)) {
+    // NVFP4 step: the prologue launch also converts the layer's weights, into slot 0
+    uint8_t* codes = reinterpret_cast<uint8_t*>(c->d_xq);
+    if (tr) cudaEventRecord(tr->e0, s);
+    if ((st = run_prologue_nvfp4(c, layer, step, x, M, ldx, codes, c->d_sf4, c->d_sx, nvfp4_w_codes(c, 0),
+                                 nvfp4_w_sf(c, layer, 0), s)) != TASQ_OK)
+      return st;
+    if (tr) cudaEventRecord(tr->e1, s);
+    if ((st = run_gemm_nvfp4(c, layer, step, codes, c->d_sf4, c->d_sx, M, y, ldy, out, 0, s)) != TASQ_OK) return st;
+    if (tr) {
+      cudaEventRecord(tr->e2, s);
+      tr->ops = 2.0 * static_cast<double>(M) * L.N * L.K;
+      tr->bytes = static_cast<double>(M) * (2.0 * L.K + L.Kp / 2.0 + L.Kp / 16.0 + 4.0) +
+                  static_cast<double>(L.N) * L.Kp * (1.0 + 0.5 + 1.0 / 16.0);
+      ++c->trace_count;
+    }
+    return TASQ_OK;
+  }
   const bool ahead = mask_ahead(c, layer, step);
   if (tr) cudaEventRecord(tr->e0, s);
   if ((st = run_prologue(c, layer, step, ahead ? std::vector<int32_t>{layer} : std::vector<int32_t>{}, x, M, ldx,
                          c->d_xq, c->d_sx, s)) != TASQ_OK)
     return st;
   if (tr) cudaEventRecord(tr->e1, s);
-  const tasq::OutKind out = c->out_dtype == TASQ_OUT_BF16 ? tasq::OutKind::BF16 : tasq::OutKind::F16;
   if ((st = run_gemm(c, layer, step, c->d_xq, c->d_sx, M, y, ldy, out, ahead, s)) != TASQ_OK) return st;
   if (tr) {
     cudaEventRecord(tr->e2, s);
@@ -547,6 +664,15 @@ tasq_status tasq_linear_forward_group(tasq_ctx* c, const void* x, int64_t M, int
   if ((st = check_device(c)) != TASQ_OK) return st;
   if (M == 0) return TASQ_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // an NVFP4 step quantizes the input differently: then every member runs as its own forward
+  for (int32_t i = 0; i < count; ++i) {
+    if (nvfp4_step(c, layers[i], step)) {
+      for (int32_t j = 0; j < count; ++j) {
+        if ((st = tasq_linear_forward(c, x, M, ldx, layers[j], step, ys[j], ldys[j], stream)) != TASQ_OK) return st;
+      }
+      return TASQ_OK;
+    }
+  }
 
   // one prologue for the shared input; it also masks, each into its own slot, the weights of
   // every member whose step drops bits
@@ -676,6 +802,77 @@ tasq_status tasq_debug_gemm(tasq_ctx* c, const int8_t* xq, const float* s_x, int
   if (M == 0) return TASQ_OK;
   const tasq::OutKind out = out_dtype == TASQ_OUT_BF16 ? tasq::OutKind::BF16 : tasq::OutKind::F16;
   return debug_gemm(c, layer, step, xq, s_x, M, y, ldy, out, static_cast<cudaStream_t>(stream));
+}
+
+tasq_status tasq_nvfp4_scale_bytes(int64_t rows, int32_t Kp, int64_t* bytes) {
+  g_last_error.clear();
+  if (bytes == nullptr) return fail(TASQ_ERR_INVALID_ARG, "bytes is NULL");
+  if (rows < 0 || Kp <= 0 || Kp % 64 != 0) return fail(TASQ_ERR_INVALID_ARG, "rows >= 0 and Kp a positive multiple of 64");
+  *bytes = tasq::nvfp4_sf_bytes(rows, Kp);
+  return TASQ_OK;
+}
+
+tasq_status tasq_debug_quantize_nvfp4(tasq_ctx* c, const void* x, int64_t M, int64_t ldx, int32_t layer, void* codes,
+                                      void* scales, float* s_x, void* stream) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  tasq_status st;
+  if ((st = check_layer(c, layer)) != TASQ_OK) return st;
+  if (M < 0 || M > 0x7fffffffLL) return fail(TASQ_ERR_INVALID_ARG, "M out of range");
+  const LayerInfo& L = c->layers[layer];
+  if ((st = check_rows(x, ldx, L.K, "x")) != TASQ_OK) return st;
+  if (codes == nullptr || !aligned16(codes) || scales == nullptr || !aligned16(scales) || s_x == nullptr)
+    return fail(TASQ_ERR_INVALID_ARG, "codes and scales must be 16-byte aligned, s_x non-NULL");
+  if ((st = check_device(c)) != TASQ_OK) return st;
+  if (M == 0) return TASQ_OK;
+  return run_prologue_nvfp4(c, layer, -1, x, M, ldx, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales), s_x,
+                            nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+tasq_status tasq_debug_nvfp4_weights(tasq_ctx* c, int32_t layer, void* codes, void* scales, void* stream) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  tasq_status st;
+  if ((st = check_layer(c, layer)) != TASQ_OK) return st;
+  if (codes == nullptr || !aligned16(codes) || scales == nullptr || !aligned16(scales))
+    return fail(TASQ_ERR_INVALID_ARG, "codes and scales must be 16-byte aligned");
+  if ((st = check_device(c)) != TASQ_OK) return st;
+  return run_prologue_nvfp4(c, layer, -1, nullptr, 0, c->layers[layer].K, nullptr, nullptr, nullptr,
+                            static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
+                            static_cast<cudaStream_t>(stream));
+}
+
+tasq_status tasq_debug_gemm_nvfp4(tasq_ctx* c, const void* codes, const void* scales, const float* s_x, int64_t M,
+                                  int32_t layer, void* y, int64_t ldy, int32_t out_kind, void* stream) {
+  g_last_error.clear();
+  if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
+  tasq_status st;
+  if ((st = check_layer(c, layer)) != TASQ_OK) return st;
+  if (M < 0 || M > 0x7fffffffLL) return fail(TASQ_ERR_INVALID_ARG, "M out of range");
+  if (out_kind != TASQ_OUT_F16 && out_kind != TASQ_OUT_BF16 && out_kind != TASQ_NVFP4_RAW_ACC)
+    return fail(TASQ_ERR_INVALID_ARG, "bad out_kind");
+  const LayerInfo& L = c->layers[layer];
+  if (codes == nullptr || !aligned16(codes) || scales == nullptr || !aligned16(scales))
+    return fail(TASQ_ERR_INVALID_ARG, "codes and scales must be 16-byte aligned");
+  if (s_x == nullptr || !aligned16(s_x)) return fail(TASQ_ERR_INVALID_ARG, "s_x must be a 16-byte aligned pointer");
+  if (out_kind == TASQ_NVFP4_RAW_ACC) {
+    if (y == nullptr || !aligned16(y) || ldy < L.N || ldy % 4 != 0)
+      return fail(TASQ_ERR_INVALID_ARG, "y must be 16-byte aligned with a row stride >= N and a multiple of 4");
+  } else if ((st = check_rows(y, ldy, L.N, "y")) != TASQ_OK) {
+    return st;
+  }
+  if ((st = check_device(c)) != TASQ_OK) return st;
+  if (M == 0) return TASQ_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the layer's weights are converted into slot 0, then the GEMM reads them from there
+  if ((st = run_prologue_nvfp4(c, layer, -1, nullptr, 0, L.K, nullptr, nullptr, nullptr, nvfp4_w_codes(c, 0),
+                               nvfp4_w_sf(c, layer, 0), s)) != TASQ_OK)
+    return st;
+  const tasq::OutKind out = out_kind == TASQ_NVFP4_RAW_ACC ? tasq::OutKind::S32
+                            : out_kind == TASQ_OUT_BF16     ? tasq::OutKind::BF16
+                                                            : tasq::OutKind::F16;
+  return run_gemm_nvfp4(c, layer, -1, static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales), s_x,
+                        M, y, ldy, out, 0, s);
 }
 
 tasq_status tasq_get_schedule(tasq_ctx* c, uint8_t* bits_host, void* stream) {

@@ -49,6 +49,44 @@ struct PrologueArgs {
 // part may be empty.
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream);
 
+// NVFP4 step (6Bit-Diffusion's stable layers): E2M1 codes with one UE4M3 scale per 16 elements
+// along K. Block scales live in 512-byte chunks, one per 128 rows x 64 elements of K; chunk
+// (row / 128) * sf_chunks + k / 64 holds the scale of row r, 16-block j of those 64 at byte
+// (r % 32) * 16 + ((r % 128) / 32) * 4 + j (the layout tcgen05.cp 32x128b.warpx4 moves into the
+// tensor memory the block-scaled MMA reads). sf_chunks = Kp4 / 64 with Kp4 = Kp rounded up to
+// 256, the K of one GEMM stage; chunks past Kp hold zero scales.
+constexpr int kNvfp4Block = 16;
+constexpr int kNvfp4Kp4 = 256;
+constexpr int kNvfp4ChunkBytes = 512;
+constexpr float kNvfp4Range = 2688.0f;   // 6 (largest E2M1) * 448 (largest E4M3)
+__host__ __device__ inline int64_t nvfp4_kp4(int64_t Kp) { return (Kp + kNvfp4Kp4 - 1) / kNvfp4Kp4 * kNvfp4Kp4; }
+__host__ __device__ inline int64_t nvfp4_sf_bytes(int64_t rows, int64_t Kp) {
+  return (rows + 127) / 128 * (nvfp4_kp4(Kp) / 64) * kNvfp4ChunkBytes;
+}
+struct Nvfp4PrologueArgs {
+  // activations: x FP16 [M, K] (row stride ldx) -> codes [M, Kp / 2], scales, s_x [M]
+  const void* x;
+  int64_t ldx;
+  int32_t K, Kp, n;
+  int64_t M;
+  uint8_t* codes;
+  uint8_t* sf;
+  float* s_x;
+  float sx_factor;     // fp32(1 / (2688 sqrt(n)))
+  // optional weight conversion in the same launch: the shared INT8 weights [N, Kp] of one layer
+  // -> NVFP4 codes [N, Kp / 2] and scales; the schedule entry bits_table[bits_index] must be 0
+  // (no check when bits_table is null)
+  const int8_t* w;
+  uint8_t* w_codes;
+  uint8_t* w_sf;
+  int32_t N;
+  const uint8_t* bits_table;
+  int32_t bits_index;
+  uint32_t* status;
+};
+cudaError_t launch_prologue_nvfp4(const Nvfp4PrologueArgs& a, cudaStream_t stream);
+
+
 enum class OutKind : int { F16 = 0, BF16 = 1, S32 = 2 };
 
 // DMPQ precision predictor: Gamma = ||out - in||_1 / ||in||_1 over FP16 [M, D] (D % 8 == 0,
@@ -93,6 +131,19 @@ struct GemmArgs {
 };
 cudaError_t launch_masked_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const CUtensorMap& tmap_y,
                                const GemmArgs& g, OutKind out, int num_sms, cudaStream_t stream);
+
+// Block-scaled NVFP4 GEMM (tcgen05 kind::mxf4nvf4), tiles of 128 channels x 128 tokens; tmap_w and
+// tmap_x cover the E2M1 codes as bytes ([N, Kp / 2] and [M, Kp / 2], boxes of 128 x 128 bytes),
+// g.num_kb = Kp4 / 256 stages, the scales in the chunked layout above (16-byte aligned). The
+// accumulators are FP32; OutKind::S32 writes their raw bits. g.bits_table may be null (no check).
+struct Nvfp4GemmArgs {
+  const uint8_t* w_sf;
+  const uint8_t* x_sf;
+  int32_t sf_chunks;   // Kp4 / 64 = 4 * g.num_kb
+};
+cudaError_t launch_gemm_nvfp4(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const CUtensorMap& tmap_y,
+                              const GemmArgs& g, const Nvfp4GemmArgs& f, OutKind out, int num_sms,
+                              cudaStream_t stream);
 
 // The same GEMM over CTA pairs (tcgen05 cta_group::2): tiles of 256 channels x 256 tokens, each
 // CTA holding 128 rows of each operand (tensor-map boxes of 128 x 128 bytes for both).
