@@ -53,6 +53,8 @@ class Workload:
     outlier_frac: float = 0.005
     # groups of block-layer indices that read the same input (one prologue feeds their GEMMs)
     shared_input: Tuple[Tuple[int, ...], ...] = ()
+    # relative_l1 schedules: the width of the stable blocks (0 = the NVFP4 step)
+    stable_bits: int = 4
 
     def forward_plan(self) -> List[Tuple[int, ...]]:
         """The block's linears in order, as tuples of block-layer indices sharing one input."""
@@ -111,9 +113,14 @@ WORKLOADS = {
         name="cogvideox", tokens=13 * 30 * 45 + 226,
         block_layers=(("qkv", 3072, 9216), ("proj", 3072, 3072), ("fc1", 3072, 12288), ("fc2", 12288, 3072)),
         blocks=42, steps=50, hadamard_n=64, schedule_kind="relative_l1"),
+    # 6Bit-Diffusion's own split on the same shapes: unstable blocks in INT8, stable ones in NVFP4
+    "cogvideox_nvfp4": Workload(
+        name="cogvideox_nvfp4", tokens=13 * 30 * 45 + 226,
+        block_layers=(("qkv", 3072, 9216), ("proj", 3072, 3072), ("fc1", 3072, 12288), ("fc2", 12288, 3072)),
+        blocks=42, steps=50, hadamard_n=64, schedule_kind="relative_l1", stable_bits=0),
 }
 
-# order of the workloads as the task lists them
+# order of the INT8 workloads as the task lists them (cogvideox_nvfp4 is the NVFP4 variant)
 WORKLOAD_ORDER = ("single", "pixart", "sana", "sdxl", "cogvideox")
 
 
@@ -163,14 +170,16 @@ def weights(wl: Workload, layer: int, seed: int = DATA_SEED) -> Tuple[np.ndarray
 
 
 def schedule(wl: Workload, seed: int = SCHEDULE_SEED) -> np.ndarray:
-    """Effective weight bits per (layer, step), uint8 [num_layers, steps], each in [1, 8].
+    """Effective weight bits per (layer, step), uint8 [num_layers, steps], each in [0, 8]
+    (0: the NVFP4 step).
 
     fixed       : the same bits for every layer at step t (single, sdxl: 8, 6, 5, 4).
     biased_high : clip(round(8 - 4 t / (T - 1) + N(0, 0.75)), 4, 8)  (pixart).
     uniform     : i.i.d. uniform over {4, ..., 8}, mean 6 (sana).
     relative_l1 : per (block, step) a synthetic relative-L1 block change Gamma ~ LogNormal(-3, 0.5);
-                  Gamma above the median of all Gamma -> 8 bits, else 4; step 0 has no previous
-                  step to measure and runs at 8; the linears of a block share its bits (cogvideox).
+                  Gamma above the median of all Gamma -> 8 bits, else stable_bits (4, or 0 for
+                  NVFP4); step 0 has no previous step to measure and runs at 8; the linears of a
+                  block share its bits (cogvideox, cogvideox_nvfp4).
     """
     L, T = wl.num_layers, wl.steps
     per_block = len(wl.block_layers)
@@ -187,7 +196,7 @@ def schedule(wl: Workload, seed: int = SCHEDULE_SEED) -> np.ndarray:
     elif wl.schedule_kind == "relative_l1":
         gamma = r.lognormal(mean=-3.0, sigma=0.5, size=(wl.blocks, T))
         thr = np.median(gamma)
-        block_bits = np.where(gamma > thr, 8, 4)
+        block_bits = np.where(gamma > thr, 8, wl.stable_bits)
         block_bits[:, 0] = 8
         bits = np.repeat(block_bits, per_block, axis=0)
     else:
