@@ -55,7 +55,8 @@ def parse_args(argv=None):
     p.add_argument("--profile-case", default=None,
                    help="workload:layer, run a few forwards of one layer (for ncu captures) and exit")
     p.add_argument("--launches", type=int, default=3)
-    p.add_argument("--bits", type=int, default=None, help="profile case: bit width (default: 5)")
+    p.add_argument("--bits", type=int, default=None,
+                   help="profile case: bit width 1..8, or 0 for the NVFP4 step (default: 5)")
     p.add_argument("--sweep-bits", default=None,
                    help="workload:layer, time one layer's prologue and GEMM at every bit width and exit")
     p.add_argument("--reps", type=int, default=20)
