@@ -272,3 +272,64 @@ def test_nvfp4_argument_errors(T):
         T.TASQ_ERR_INVALID_ARG
     assert err(T.tasq_nvfp4_scale_bytes, 8, 100) == T.TASQ_ERR_INVALID_ARG
     assert err(T.tasq_set_schedule, ctx, np.array([[9]], np.uint8), _stream()) == T.TASQ_ERR_INVALID_ARG
+
+
+def _nvfp4_tol(r, s_w, Kp):
+    return (_terms_bound(r["ca"], r["sa"], r["cw"], r["sw"], Kp) * r["s_x"][:, None] * s_w[None, :] * 1.0001 +
+            np.abs(r["y"]) * (2.0 ** -11 + 2.0 ** -21) + 2.0 ** -24)
+
+
+def test_nvfp4_in_a_group_forward(T):
+    """A group whose step is NVFP4 for one member runs every member as its own forward: each
+    output equals that member's oracle linear (NVFP4 or INT8)."""
+    rng = np.random.default_rng(37)
+    n, K, M = 64, 1280, 300
+    shapes = [1280, 640, 896]
+    layers = []
+    for N in shapes:
+        w = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+        s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+        layers.append((N, K, w, s_w))
+    ctx = _ctx(T, layers, 1, n, M)
+    T.tasq_set_schedule(ctx, np.array([[8], [0], [5]], np.uint8), _stream())
+    x = _acts(rng, M, K)
+    ys = [torch.empty((M, N), dtype=torch.float16, device="cuda") for N in shapes]
+    T.tasq_linear_forward_group(ctx, _dev(x), M, K, [0, 1, 2], 0, ys, list(shapes), _stream())
+    torch.cuda.synchronize()
+    for (N, _, w, s_w), y, b in zip(layers, ys, (8, 0, 5)):
+        got = y.float().cpu().numpy().astype(np.float64)
+        if b == 0:
+            r = oracle.nvfp4_linear(x, w, s_w, n)
+            assert np.all(np.abs(got - r["y"]) <= _nvfp4_tol(r, s_w, K)), "NVFP4 member"
+        else:
+            ref = oracle.masked_linear(x, w, s_w, b, n)["y"]
+            assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 1e-3, f"INT8 member, bits {b}"
+    assert T.tasq_get_device_status(ctx) == 0
+
+
+def test_nvfp4_forward_replays_from_a_cuda_graph(T):
+    """NVFP4 and INT8 forwards captured in one CUDA graph replay to the bits of the direct launches."""
+    rng = np.random.default_rng(43)
+    n, K, N, M = 64, 1152, 1152, 512
+    x = _acts(rng, M, K)
+    w = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+    ctx = _ctx(T, [(N, K, w, s_w)], 2, n, M)
+    T.tasq_set_schedule(ctx, np.array([[0, 6]], np.uint8), _stream())
+    xd = _dev(x)
+    eager = [torch.empty((M, N), dtype=torch.float16, device="cuda") for _ in range(2)]
+    for step in range(2):
+        T.tasq_linear_forward(ctx, xd, M, K, 0, step, eager[step], N, _stream())
+    torch.cuda.synchronize()
+    replay = [torch.zeros((M, N), dtype=torch.float16, device="cuda") for _ in range(2)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for step in range(2):
+            T.tasq_linear_forward(ctx, xd, M, K, 0, step, replay[step], N, torch.cuda.current_stream())
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(eager, replay):
+        assert torch.equal(a, b)
+    assert T.tasq_get_schedule(ctx).reshape(-1).tolist() == [0, 6], "the table keeps the NVFP4 entry"
+    assert T.tasq_get_device_status(ctx) == 0
