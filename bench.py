@@ -64,6 +64,8 @@ def parse_args(argv=None):
                    help="GEMM kernel: 0 automatic, 1 one CTA per tile, 2 CTA pairs")
     p.add_argument("--mask-mode", type=int, default=0, choices=[0, 1, 2],
                    help="LSB mask: 0 automatic, 1 inside the GEMM on every tile, 2 once ahead in the prologue launch")
+    p.add_argument("--bitplanes", default=None,
+                   help="workload:layer -- time the bit-plane formulation against the masked dense GEMM")
     p.add_argument("--gemm-shape", default=None,
                    help="M,N,K: time the GEMM alone on given codes (one JSON line) and exit")
     p.add_argument("--graph", action="store_true",
@@ -456,6 +458,66 @@ def gemm_shape(args):
     return 0
 
 
+def bitplanes(args):
+    """The bit-plane formulation measured (TASQ's Temporal-Precision Engine streams only the kept
+    weight bit planes, TASQ technical summary section 2). On B200 the only integer tensor-core
+    MMA is kind::i8, so a plane P_i of the weights (entries 0 or 1, the sign plane 0 or -1) costs
+    one INT8 GEMM, and b kept planes cost b of them (plus the sum of the partial products). This
+    times, at one layer's full shape, the masked dense GEMM at several widths and the same GEMM on
+    a single bit plane, all on identical activation codes."""
+    import torch
+    import timestep_adaptive_bit_b200 as T
+    name, _, lname = args.bitplanes.partition(":")
+    wl = workloads.WORKLOADS[name]
+    j = [n for n, _, _ in wl.block_layers].index(lname or wl.block_layers[0][0])
+    _, K, N = wl.layer_shape(j)
+    M = wl.tokens
+    dev = torch.device("cuda:0")
+    s = torch.cuda.current_stream()
+    w, s_w = workloads.weights_torch(wl, j, dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    Kp = w.shape[1]
+    q = torch.randint(-127, 128, (M, Kp), dtype=torch.int8, device=dev, generator=g)
+    s_x = torch.rand((M,), device=dev, generator=g) + 0.5
+    y = torch.empty((M, N), dtype=torch.float16, device=dev)
+
+    def timed(ctx, step):
+        for _ in range(3):
+            T.tasq_debug_gemm(ctx, q, s_x, M, 0, step, y, N, T.TASQ_OUT_F16, s)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(args.reps):
+            T.tasq_debug_gemm(ctx, q, s_x, M, 0, step, y, N, T.TASQ_OUT_F16, s)
+        e1.record(s)
+        torch.cuda.synchronize()
+        assert T.tasq_get_device_status(ctx) == 0
+        return 1e3 * e0.elapsed_time(e1) / args.reps
+
+    widths = (8, 6, 4, 2, 1)
+    ctx = T.tasq_linear_create([(N, K, w, s_w)], len(widths), wl.hadamard_n, M, T.TASQ_OUT_F16, s)
+    T.tasq_set_schedule(ctx, np.array([widths], np.uint8), s)
+    T.tasq_debug_set_mask_mode(ctx, 2)        # the weights masked once ahead, as in a forward
+    dense = {b: timed(ctx, i) for i, b in enumerate(widths)}
+    T.tasq_linear_destroy(ctx)
+    planes = {}
+    for name_p, plane in (("plane_3", ((w.to(torch.int16) >> 3) & 1).to(torch.int8)),
+                          ("sign_plane", -((w.to(torch.int16) >> 7) & 1).to(torch.int8))):
+        ctx = T.tasq_linear_create([(N, K, plane.contiguous(), s_w)], 1, wl.hadamard_n, M, T.TASQ_OUT_F16, s)
+        planes[name_p] = timed(ctx, 0)
+        T.tasq_linear_destroy(ctx)
+    t_plane = max(planes.values())
+    out = {"bitplanes": args.bitplanes, "M": M, "N": N, "K": K,
+           "dense_masked_us": {str(b): round(t, 2) for b, t in dense.items()},
+           "one_plane_us": {k: round(v, 2) for k, v in planes.items()},
+           "bit_plane_gemm_us_lower_bound": {str(b): round(b * t_plane, 2) for b in widths},
+           "note": "b kept planes = b INT8 GEMMs on 0/1 planes; the lower bound leaves out summing them"}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def sweep_bits(args):
     """Per-bit-width timing of one layer at full size (CUDA-event trace of each kernel)."""
     import torch
@@ -521,6 +583,8 @@ def main(argv=None):
         return sweep_bits(args)
     if args.gemm_shape:
         return gemm_shape(args)
+    if args.bitplanes:
+        return bitplanes(args)
 
     dist = None
     if world > 1:
