@@ -1,7 +1,8 @@
 """Full-size parity: every distinct layer shape of every workload at its full token count, run
 through tasq_linear_forward exactly as the bench launches it, checked on a seeded sample of
 token rows (plus the whole last, ragged token tile) against the oracle computed row by row.
-Each layer runs at the lowest bit width its schedule gives it and at 8 bits."""
+Each layer runs at every bit width its schedule gives it (a (layer, step) result depends on the
+step only through that width), and the NVFP4 workload's layers also in their NVFP4 step."""
 import numpy as np
 import pytest
 
@@ -38,10 +39,11 @@ def test_fullsize_workload(T, name):
         w, s_w = workloads.weights(wl, j)
         layers.append((N, K, w, s_w))
         xs.append(workloads.activations(wl, j))
-    low = [int(sched[j::len(wl.block_layers)].min()) for j in picked]
-    table = np.array([[8, b] for b in low], np.uint8)
+    # step t of the test table runs width 8 - t: every width a layer's schedule uses is one step
+    widths = [sorted({int(v) for v in sched[j::len(wl.block_layers)].ravel()}, reverse=True) for j in picked]
+    table = np.array([[8 - t for t in range(8)] for _ in picked], np.uint8)
     s = torch.cuda.current_stream()
-    ctx = T.tasq_linear_create(layers, 2, n, M, 0, s)
+    ctx = T.tasq_linear_create(layers, 8, n, M, 0, s)
     T.tasq_set_schedule(ctx, table, s)
     rows = workloads.sample_rows(M)
     for li, ((N, K, w, s_w), x) in enumerate(zip(layers, xs)):
@@ -58,7 +60,8 @@ def test_fullsize_workload(T, name):
         assert d.max() <= 1 and d.astype(bool).mean() <= 1e-3
         assert np.all(np.abs(sx.cpu().numpy()[rows] - sx_ref) <= 1e-6 * np.abs(sx_ref))
         del xq
-        for step, bits in ((0, 8), (1, low[li])):
+        for bits in widths[li]:
+            step = 8 - bits
             y = torch.empty((M, N), dtype=torch.float16, device="cuda")
             T.tasq_linear_forward(ctx, xd, M, K, li, step, y, N, s)
             torch.cuda.synchronize()
@@ -72,3 +75,36 @@ def test_fullsize_workload(T, name):
         del xd
     assert T.tasq_get_device_status(ctx) == 0
     T.tasq_linear_destroy(ctx)
+
+
+def test_fullsize_nvfp4_workload(T):
+    """CogVideoX with its stable blocks in NVFP4: every distinct layer shape at the full 17776
+    tokens in its NVFP4 step, on sampled rows, within the FP32 accumulation bound."""
+    wl = workloads.WORKLOADS["cogvideox_nvfp4"]
+    M, n = wl.tokens, wl.hadamard_n
+    assert (workloads.schedule(wl) == 0).any()
+    rows = workloads.sample_rows(M)
+    s = torch.cuda.current_stream()
+    seen = set()
+    for j, (lname, K, N) in enumerate(wl.block_layers):
+        if (K, N) in seen:
+            continue
+        seen.add((K, N))
+        w, s_w = workloads.weights(wl, j)
+        x = workloads.activations(wl, j)
+        ctx = T.tasq_linear_create([(N, K, w, s_w)], 1, n, M, 0, s)
+        T.tasq_set_schedule(ctx, np.array([[0]], np.uint8), s)
+        xd = torch.from_numpy(x).cuda()
+        y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+        T.tasq_linear_forward(ctx, xd, M, K, 0, 0, y, N, s)
+        torch.cuda.synchronize()
+        got = y[torch.from_numpy(rows).cuda()].float().cpu().numpy().astype(np.float64)
+        r = oracle.nvfp4_linear(x[rows], w, s_w, n)
+        Kp = oracle.padded_k(K, n)
+        bound = (Kp * 2.0 ** -24 * oracle.nvfp4_abs_terms(r["ca"], r["sa"], r["cw"], r["sw"]) * 1.0001 *
+                 r["s_x"][:, None] * s_w[None, :] + np.abs(r["y"]) * (2.0 ** -11 + 2.0 ** -21) + 2.0 ** -24)
+        assert np.all(np.abs(got - r["y"]) <= bound), lname
+        assert np.all(np.isfinite(y.float().cpu().numpy())), "non-finite output"
+        assert T.tasq_get_device_status(ctx) == 0
+        T.tasq_linear_destroy(ctx)
+        del xd, y
