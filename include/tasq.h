@@ -200,8 +200,12 @@ tasq_status tasq_get_schedule(tasq_ctx* ctx, uint8_t* bits_host, void* stream);
  * over the previous step, Gamma = ||out - in||_1 / ||in||_1, picks the bit width of the block's
  * linears for `step`: bits[layer][step] = Gamma > tau ? bits_unstable : bits_stable for every
  * layer in `layers`. When ||in||_1 = 0, Gamma is +inf (or 0 if the output is zero as well) and
- * the layers take bits_unstable. The pages compress stable layers to NVFP4; here the stable
- * width is an LSB-masked width of the same INT8 buffer.
+ * the layers take bits_unstable. Each width is an INT8 width 1..8 or TASQ_NVFP4 (0): the pages
+ * keep unstable layers in INT8 and compress stable ones to NVFP4 (bits_unstable = 8,
+ * bits_stable = TASQ_NVFP4). When one of the two is NVFP4, later forwards of these (layer, step)
+ * entries launch both the INT8 and the NVFP4 kernels; each reads the device table and the one
+ * whose format was not chosen returns at once, so the choice needs no host round trip and holds
+ * inside a captured CUDA graph as well.
  *   block_in, block_out : device FP16 [M, D], the block's input and output at the previous
  *                         step, row strides ld_in / ld_out (elements, >= D, % 8 == 0), 16-byte
  *                         aligned; D % 8 == 0. Neither is modified.
@@ -234,7 +238,7 @@ tasq_status tasq_dmpq_update(tasq_ctx* ctx, const void* block_in, int64_t ld_in,
  * nibble; block scales use 512-byte chunks, one per 128 rows x 64 elements of K, in which row r
  * and 16-block j sit at byte (r % 32) * 16 + ((r % 128) / 32) * 4 + j, the chunks of a 128-row
  * group in K order; K is padded with zero scales to a multiple of 256.
- * tasq_linear_forward_noalloc and tasq_dmpq_update stay INT8-only.
+ * tasq_linear_forward_noalloc stays INT8-only.
  */
 #define TASQ_NVFP4 0
 #define TASQ_NVFP4_RAW_ACC 2   /* out_kind of tasq_debug_gemm_nvfp4: raw FP32 accumulators */

@@ -164,7 +164,61 @@ def test_argument_errors(T):
     assert err(z, 32, z, 32, 4, 32, [2], 0, 0.5, 8, 4, None, _s()) == E          # layer range
     assert err(z, 32, z, 32, 4, 32, [0], 2, 0.5, 8, 4, None, _s()) == E          # step range
     assert err(z, 32, z, 32, 4, 32, [0], 0, 0.5, 9, 4, None, _s()) == E          # bits
+    assert err(z, 32, z, 32, 4, 32, [0], 0, 0.5, 8, -1, None, _s()) == E         # bits
     assert err(z, 32, z, 32, 4, 32, [0], 0, float("nan"), 8, 4, None, _s()) == E
     assert err(z.data_ptr() + 2, 32, z, 32, 4, 32, [0], 0, 0.5, 8, 4, None, _s()) == E   # alignment
     assert err(z, 30, z, 32, 4, 32, [0], 0, 0.5, 8, 4, None, _s()) == E          # row stride
     assert np.all(T.tasq_get_schedule(ctx, _s()) == 8), "a rejected call changes nothing"
+
+
+def _nvfp4_close(got, x, w, s_w, n):
+    r = oracle.nvfp4_linear(x, w, s_w, n)
+    Kp = oracle.padded_k(x.shape[1], n)
+    bound = (Kp * 2.0 ** -24 * oracle.nvfp4_abs_terms(r["ca"], r["sa"], r["cw"], r["sw"]) * 1.0001 *
+             r["s_x"][:, None] * s_w[None, :] + np.abs(r["y"]) * (2.0 ** -11 + 2.0 ** -21) + 2.0 ** -24)
+    return np.all(np.abs(got - r["y"]) <= bound)
+
+
+def test_predictor_chooses_int8_or_nvfp4_on_the_device(T):
+    """6Bit-Diffusion's split: unstable blocks INT8, stable ones NVFP4, decided on the device. The
+    forward after the predictor launches both paths gated on the table; the output is the INT8
+    result when Gamma > tau and the NVFP4 result otherwise, with no host round trip, also from a
+    CUDA graph captured once and replayed after the decision changed."""
+    rng = np.random.default_rng(23)
+    M, K, N, n = 384, 1152, 896, 64
+    x = (rng.standard_normal((M, K))).astype(np.float16)
+    w = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+    ctx = T.tasq_linear_create([(N, K, w, s_w)], 1, n, M, T.TASQ_OUT_F16, _s())
+    x_in, x_out, din, dout, ld = _pair(rng, M, K)
+    gamma = oracle.dmpq_gamma(x_in, x_out)
+    xd = torch.from_numpy(x).cuda()
+    ref8 = oracle.masked_linear(x, w, s_w, 8, n)["y"]
+    # direct launches: stable -> NVFP4, then unstable -> INT8
+    for tau, want in ((gamma * 2, "nvfp4"), (gamma / 2, "int8")):
+        T.tasq_dmpq_update(ctx, din, ld, dout, ld, M, K, [0], 0, tau, 8, T.TASQ_NVFP4, None, _s())
+        y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+        T.tasq_linear_forward(ctx, xd, M, K, 0, 0, y, N, _s())
+        torch.cuda.synchronize()
+        got = y.float().cpu().numpy().astype(np.float64)
+        assert int(T.tasq_get_schedule(ctx, _s())[0, 0]) == (0 if want == "nvfp4" else 8)
+        if want == "nvfp4":
+            assert _nvfp4_close(got, x, w, s_w, n), "NVFP4 chosen on the device"
+        else:
+            assert np.all(np.abs(got - ref8) <= F16_REL * np.abs(ref8) + ABS_TINY), "INT8 chosen on the device"
+    # one captured graph of predictor + forward, replayed with tau moved between replays
+    y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+    T.tasq_dmpq_update(ctx, din, ld, dout, ld, M, K, [0], 0, gamma * 2, 8, T.TASQ_NVFP4, None, _s())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        T.tasq_linear_forward(ctx, xd, M, K, 0, 0, y, N, torch.cuda.current_stream())
+    for tau, want in ((gamma * 2, "nvfp4"), (gamma / 2, "int8"), (gamma * 2, "nvfp4")):
+        T.tasq_dmpq_update(ctx, din, ld, dout, ld, M, K, [0], 0, tau, 8, T.TASQ_NVFP4, None, _s())
+        g.replay()
+        torch.cuda.synchronize()
+        got = y.float().cpu().numpy().astype(np.float64)
+        if want == "nvfp4":
+            assert _nvfp4_close(got, x, w, s_w, n), "graph replay, NVFP4"
+        else:
+            assert np.all(np.abs(got - ref8) <= F16_REL * np.abs(ref8) + ABS_TINY), "graph replay, INT8"
+    assert T.tasq_get_device_status(ctx) == 0

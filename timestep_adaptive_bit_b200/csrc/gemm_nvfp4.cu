@@ -77,6 +77,7 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   ptx::grid_dep_launch_dependents();
+  if (g.bits_table != nullptr && gated_out(g.gate, g.bits_table, g.bits_index)) return;
 
   // the schedule entry of an NVFP4 step is 0
   if (threadIdx.x == 0 && g.bits_table != nullptr && g.bits_table[g.bits_index] != 0)

@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
   const int lane = threadIdx.x & 31;
   // the next kernel of the stream may be scheduled; it waits for this one before reading
   ptx::grid_dep_launch_dependents();
+  if (gated_out(g.gate, g.bits_table, g.bits_index)) return;
 
   // schedule lookup: the step's bit width for this layer
   int bits = g.bits_table[g.bits_index];

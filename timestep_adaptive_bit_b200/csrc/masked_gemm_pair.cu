@@ -80,6 +80,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   // the next kernel of the stream may be scheduled; it waits for this one before reading
   ptx::grid_dep_launch_dependents();
+  if (gated_out(g.gate, g.bits_table, g.bits_index)) return;   // uniform: both CTAs of a pair leave
   const uint32_t rank = ptx::cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   const bool leader = rank == 0;

@@ -240,6 +240,7 @@ __device__ __forceinline__ void weight_pass(const PrologueArgs& a, int64_t cta, 
 template <int LANES, bool VEC32, int MAXT, int MINB>
 __global__ void __launch_bounds__(MAXT, MINB)
     prologue_kernel(const PrologueArgs a, const int rows_per_cta, const int row_ctas) {
+  if (gated_out(a.gate, a.bits_table, a.gate_index)) return;
   if (static_cast<int>(blockIdx.x) >= row_ctas) {
     weight_pass(a, blockIdx.x - row_ctas, gridDim.x - row_ctas);
     return;
@@ -411,6 +412,7 @@ __device__ __forceinline__ void nvfp4_weight_pass(const Nvfp4PrologueArgs& a, in
 template <int LANES, int MAXT, int MINB>
 __global__ void __launch_bounds__(MAXT, MINB)
     prologue_nvfp4_kernel(const Nvfp4PrologueArgs a, const int rows_per_cta, const int row_ctas) {
+  if (gated_out(a.gate, a.gate_table, a.gate_index)) return;
   if (static_cast<int>(blockIdx.x) >= row_ctas) {
     nvfp4_weight_pass(a, blockIdx.x - row_ctas, gridDim.x - row_ctas);
     return;
@@ -531,6 +533,7 @@ __device__ __forceinline__ bool all_compute(bool p, int T) {
 template <int LANES>
 __global__ void __launch_bounds__(kFedMaxCompute + 32, 1)
     prologue_fed_kernel(const PrologueArgs a, const FedGeom geo) {
+  if (gated_out(a.gate, a.bits_table, a.gate_index)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const uint32_t sbase = ptx::smem_addr(smem);

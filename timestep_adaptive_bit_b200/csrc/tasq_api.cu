@@ -148,6 +148,9 @@ struct tasq_ctx {
   // places read the device table and give the same result for every bit width, so a device table
   // that is newer or older than this copy changes no result
   std::vector<uint8_t> bits_host;
+  // entries the on-device predictor may have set to either an INT8 width (kept in bits_host) or
+  // NVFP4: forwards of such an entry launch both paths, gated on the device table
+  std::vector<uint8_t> maybe_nvfp4;
   int8_t* d_wk = nullptr;              // masked copies: wk_slots slots of wk_slot_bytes each
   size_t wk_slot_bytes = 0;            // largest N x Kp, rounded up to 1024
   int32_t wk_slots = 0;                // min(num_layers, TASQ_GROUP_MAX)
@@ -249,7 +252,8 @@ void add_weight_pass(tasq::PrologueArgs& a, const tasq_ctx* c, int32_t layer, in
 // `masked` lists up to kMaxWeightSegments layers whose weights the same launch masks, layer
 // masked[i] into masked-weight slot i.
 tasq_status run_prologue(tasq_ctx* c, int32_t layer, int32_t step, const std::vector<int32_t>& masked, const void* x,
-                         int64_t M, int64_t ldx, int8_t* xq, float* sx, cudaStream_t s) {
+                         int64_t M, int64_t ldx, int8_t* xq, float* sx, cudaStream_t s,
+                         int32_t gate = tasq::kGateNone) {
   const LayerInfo& L = c->layers[layer];
   tasq::PrologueArgs a{};
   for (size_t i = 0; i < masked.size(); ++i) add_weight_pass(a, c, masked[i], step, static_cast<int32_t>(i));
@@ -266,6 +270,9 @@ tasq_status run_prologue(tasq_ctx* c, int32_t layer, int32_t step, const std::ve
   a.wait_limit_ns = c->wait_limit_ns;
   a.num_sms = c->num_sms;
   a.variant = c->prologue_mode;
+  a.bits_table = c->d_bits;
+  a.gate = gate;
+  a.gate_index = layer * c->num_steps + step;
   g_last_error.clear();
   cudaError_t e = tasq::launch_prologue(a, s);
   if (e != cudaSuccess) {
@@ -280,6 +287,11 @@ bool nvfp4_step(const tasq_ctx* c, int32_t layer, int32_t step) {
   return c->bits_host[static_cast<size_t>(layer) * c->num_steps + step] == 0;
 }
 
+// Whether the device may have chosen either format for this entry (see maybe_nvfp4).
+bool either_format(const tasq_ctx* c, int32_t layer, int32_t step) {
+  return c->maybe_nvfp4[static_cast<size_t>(layer) * c->num_steps + step] != 0;
+}
+
 // The NVFP4 weights of a layer live in masked-weight slot `slot`: codes [N, Kp / 2] at its start,
 // block scales from the next 512-byte boundary.
 uint8_t* nvfp4_w_codes(const tasq_ctx* c, int32_t slot) { return reinterpret_cast<uint8_t*>(wk_slot(c, slot)); }
@@ -292,7 +304,7 @@ uint8_t* nvfp4_w_sf(const tasq_ctx* c, int32_t layer, int32_t slot) {
 // layer's weights converted into w_codes / w_sf. step < 0: no schedule check.
 tasq_status run_prologue_nvfp4(tasq_ctx* c, int32_t layer, int32_t step, const void* x, int64_t M, int64_t ldx,
                                uint8_t* codes, uint8_t* sf, float* sx, uint8_t* w_codes, uint8_t* w_sf,
-                               cudaStream_t s) {
+                               cudaStream_t s, int32_t gate = tasq::kGateNone) {
   const LayerInfo& L = c->layers[layer];
   tasq::Nvfp4PrologueArgs a{};
   a.x = x;
@@ -315,6 +327,11 @@ tasq_status run_prologue_nvfp4(tasq_ctx* c, int32_t layer, int32_t step, const v
     if (step < 0) a.bits_table = nullptr;
   }
   a.status = c->d_status;
+  if (step >= 0 && gate != tasq::kGateNone) {
+    a.gate = gate;
+    a.gate_table = c->d_bits;
+    a.gate_index = layer * c->num_steps + step;
+  }
   cudaError_t e = tasq::launch_prologue_nvfp4(a, s);
   if (e != cudaSuccess) return fail_cuda(e, "NVFP4 prologue launch");
   return TASQ_OK;
@@ -324,7 +341,7 @@ tasq_status run_prologue_nvfp4(tasq_ctx* c, int32_t layer, int32_t step, const v
 // step < 0: no schedule check. out S32 writes the raw FP32 accumulators.
 tasq_status run_gemm_nvfp4(tasq_ctx* c, int32_t layer, int32_t step, const uint8_t* codes, const uint8_t* sf,
                            const float* sx, int64_t M, void* y, int64_t ldy, tasq::OutKind out, int32_t slot,
-                           cudaStream_t s) {
+                           cudaStream_t s, int32_t gate = tasq::kGateNone) {
   const LayerInfo& L = c->layers[layer];
   const int64_t kp4 = tasq::nvfp4_kp4(L.Kp);
   CUtensorMap tw, tx, ty;
@@ -353,6 +370,7 @@ tasq_status run_gemm_nvfp4(tasq_ctx* c, int32_t layer, int32_t step, const uint8
   g.ldy = ldy;
   g.status = c->d_status;
   g.wait_limit_ns = c->wait_limit_ns;
+  g.gate = step < 0 ? tasq::kGateNone : gate;
   tasq::Nvfp4GemmArgs f{};
   f.w_sf = nvfp4_w_sf(c, layer, slot);
   f.x_sf = sf;
@@ -392,7 +410,8 @@ namespace {
 
 // GEMM of (layer, step). premasked: the weights come masked from masked-weight slot `slot`.
 tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq, const float* sx, int64_t M,
-                     void* y, int64_t ldy, tasq::OutKind out, bool premasked, cudaStream_t s, int32_t slot = 0) {
+                     void* y, int64_t ldy, tasq::OutKind out, bool premasked, cudaStream_t s, int32_t slot = 0,
+                     int32_t gate = tasq::kGateNone) {
   const LayerInfo& L = c->layers[layer];
   const bool pair = c->gemm_mode == 2 || (c->gemm_mode == 0 && tasq::gemm_use_pair(M, L.N, c->num_sms));
   const int tile_tok = pair ? tasq::kGemmPairTile : tasq::kGemmTileTok;
@@ -423,6 +442,7 @@ tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq,
   g.status = c->d_status;
   g.wait_limit_ns = c->wait_limit_ns;
   g.premasked = premasked ? 1 : 0;
+  g.gate = gate;
   CUtensorMap tw = premasked ? c->tmap_wk[layer] : c->tmap_w[layer];
   if (premasked && slot != 0) {
     st = make_tmap_u8(&tw, wk_slot(c, slot), static_cast<uint64_t>(L.Kp), static_cast<uint64_t>(L.N),
@@ -545,6 +565,7 @@ tasq_status tasq_linear_create(tasq_ctx** out, const tasq_layer_desc* layers, in
 
   if ((e = cudaMemsetAsync(c->d_bits, 8, table, s)) != cudaSuccess) return bail(e, "cudaMemsetAsync(schedule)");
   c->bits_host.assign(table, 8);
+  c->maybe_nvfp4.assign(table, 0);
   if ((e = cudaMemsetAsync(c->d_status, 0, sizeof(uint32_t), s)) != cudaSuccess) return bail(e, "cudaMemsetAsync(status)");
   for (int32_t l = 0; l < num_layers; ++l) {
     const LayerInfo& L = info[l];
@@ -589,6 +610,7 @@ tasq_status tasq_set_schedule(tasq_ctx* c, const uint8_t* bits_host, void* strea
   cudaError_t e = cudaMemcpyAsync(c->d_bits, bits_host, table, cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e, "copy of schedule");
   c->bits_host.assign(bits_host, bits_host + table);
+  c->maybe_nvfp4.assign(table, 0);
   return TASQ_OK;
 }
 
@@ -609,6 +631,32 @@ tasq_status tasq_linear_forward(tasq_ctx* c, const void* x, int64_t M, int64_t l
 
   TraceRec* tr = c->trace_count < c->trace_cap ? &c->trace[c->trace_count] : nullptr;
   const tasq::OutKind out = c->out_dtype == TASQ_OUT_BF16 ? tasq::OutKind::BF16 : tasq::OutKind::F16;
+  if (either_format(c, layer, step)) {
+    // the predictor decided on the device: both paths are launched, each gated on the table, and
+    // exactly one of them runs (the INT8 width the host knows of is bits_host's entry)
+    uint8_t* codes4 = reinterpret_cast<uint8_t*>(c->d_xq);
+    const bool ahead = mask_ahead(c, layer, step);
+    if (tr) cudaEventRecord(tr->e0, s);
+    if ((st = run_prologue(c, layer, step, ahead ? std::vector<int32_t>{layer} : std::vector<int32_t>{}, x, M, ldx,
+                           c->d_xq, c->d_sx, s, tasq::kGateInt8)) != TASQ_OK)
+      return st;
+    if ((st = run_prologue_nvfp4(c, layer, step, x, M, ldx, codes4, c->d_sf4, c->d_sx, nvfp4_w_codes(c, 0),
+                                 nvfp4_w_sf(c, layer, 0), s, tasq::kGateNvfp4)) != TASQ_OK)
+      return st;
+    if (tr) cudaEventRecord(tr->e1, s);
+    if ((st = run_gemm(c, layer, step, c->d_xq, c->d_sx, M, y, ldy, out, ahead, s, 0, tasq::kGateInt8)) != TASQ_OK)
+      return st;
+    if ((st = run_gemm_nvfp4(c, layer, step, codes4, c->d_sf4, c->d_sx, M, y, ldy, out, 0, s, tasq::kGateNvfp4)) !=
+        TASQ_OK)
+      return st;
+    if (tr) {
+      cudaEventRecord(tr->e2, s);
+      tr->ops = 2.0 * static_cast<double>(M) * L.N * L.K;
+      tr->bytes = static_cast<double>(M) * (2.0 * L.K + L.Kp + 4.0) + (ahead ? 2.0 * L.N * L.Kp : 0.0);
+      ++c->trace_count;
+    }
+    return TASQ_OK;
+  }
   if (nvfp4_step(c, layer, step)) {
     // NVFP4 step: the prologue launch also converts the layer's weights, into slot 0
     uint8_t* codes = reinterpret_cast<uint8_t*>(c->d_xq);
@@ -666,7 +714,7 @@ tasq_status tasq_linear_forward_group(tasq_ctx* c, const void* x, int64_t M, int
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // an NVFP4 step quantizes the input differently: then every member runs as its own forward
   for (int32_t i = 0; i < count; ++i) {
-    if (nvfp4_step(c, layers[i], step)) {
+    if (nvfp4_step(c, layers[i], step) || either_format(c, layers[i], step)) {
       for (int32_t j = 0; j < count; ++j) {
         if ((st = tasq_linear_forward(c, x, M, ldx, layers[j], step, ys[j], ldys[j], stream)) != TASQ_OK) return st;
       }
@@ -899,8 +947,8 @@ tasq_status tasq_dmpq_update(tasq_ctx* c, const void* block_in, int64_t ld_in, c
     return fail(TASQ_ERR_INVALID_ARG, "need 1 to TASQ_DMPQ_MAX_LAYERS layer indices");
   for (int32_t i = 0; i < num_block_layers; ++i)
     if ((st = check_layer(c, layers[i])) != TASQ_OK) return st;
-  if (bits_unstable < 1 || bits_unstable > 8 || bits_stable < 1 || bits_stable > 8)
-    return fail(TASQ_ERR_INVALID_ARG, "bit widths must be in [1, 8]");
+  if (bits_unstable < 0 || bits_unstable > 8 || bits_stable < 0 || bits_stable > 8)
+    return fail(TASQ_ERR_INVALID_ARG, "widths must be in [0, 8] (0: NVFP4)");
   if (!(tau == tau)) return fail(TASQ_ERR_INVALID_ARG, "tau is NaN");
   if (M < 0 || M > 0x7fffffffLL) return fail(TASQ_ERR_INVALID_ARG, "M out of range");
   if (D < 8 || D % 8 != 0) return fail(TASQ_ERR_INVALID_ARG, "D must be a positive multiple of 8");
@@ -929,11 +977,21 @@ tasq_status tasq_dmpq_update(tasq_ctx* c, const void* block_in, int64_t ld_in, c
   a.gamma_out = gamma_out;
   cudaError_t e = tasq::launch_dmpq(a, c->d_dmpq, c->d_dmpq_arrived, c->num_sms, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e, "predictor launch");
-  // the host copy of the table only steers where the mask is applied: take the narrower width,
-  // so that a dropped bit is masked once ahead of the GEMM whichever way the device decides
-  const uint8_t hint = static_cast<uint8_t>(bits_unstable < bits_stable ? bits_unstable : bits_stable);
-  for (int32_t i = 0; i < num_block_layers; ++i)
-    c->bits_host[static_cast<size_t>(layers[i]) * c->num_steps + step] = hint;
+  // the host copy of the table steers where the mask is applied and which kernels a forward
+  // launches. Both widths INT8: take the narrower one, so that a dropped bit is masked once ahead
+  // of the GEMM whichever way the device decides. One of them NVFP4: keep the INT8 one and mark
+  // the entry, so that its forwards launch both paths gated on the table. Both NVFP4: NVFP4.
+  const bool f4u = bits_unstable == 0, f4s = bits_stable == 0;
+  const uint8_t hint = static_cast<uint8_t>(f4u && f4s ? 0
+                                            : f4u       ? bits_stable
+                                            : f4s       ? bits_unstable
+                                            : (bits_unstable < bits_stable ? bits_unstable : bits_stable));
+  const uint8_t either = (f4u != f4s) ? 1 : 0;
+  for (int32_t i = 0; i < num_block_layers; ++i) {
+    const size_t entry = static_cast<size_t>(layers[i]) * c->num_steps + step;
+    c->bits_host[entry] = hint;
+    c->maybe_nvfp4[entry] = either;
+  }
   return TASQ_OK;
 }
 

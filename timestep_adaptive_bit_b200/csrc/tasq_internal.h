@@ -44,10 +44,27 @@ struct PrologueArgs {
   int32_t num_sms;
   int32_t variant;    // 0: bulk-fed for long launches, else direct; 1: always direct;
                       // 2: bulk-fed wherever its layout fits
+  int32_t gate;       // kGateNone, or kGateInt8: the launch steps aside when the schedule entry
+  int32_t gate_index; //   bits_table[gate_index] is 0 (an NVFP4 step decided on the device)
 };
 // Launches the activation rows (M > 0) and the weight pass (num_w > 0) as one grid; either
 // part may be empty.
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream);
+
+// Gated launches. When the on-device predictor may pick either format for a (layer, step), a
+// forward launches both the INT8 and the NVFP4 kernels; each reads the schedule entry first and,
+// if the step is not its format, waits for the kernel before it (so the launches after it still
+// see that kernel's results) and returns without touching memory.
+constexpr int32_t kGateNone = 0;
+constexpr int32_t kGateInt8 = 1;    // run only if the entry is 1..8
+constexpr int32_t kGateNvfp4 = 2;   // run only if the entry is 0
+__device__ __forceinline__ bool gated_out(int32_t gate, const uint8_t* table, int32_t index) {
+  if (gate == kGateNone) return false;
+  const bool nvfp4 = table[index] == 0;
+  const bool skip = gate == kGateInt8 ? nvfp4 : !nvfp4;
+  if (skip) asm volatile("griddepcontrol.wait;" ::: "memory");
+  return skip;
+}
 
 // NVFP4 step (6Bit-Diffusion's stable layers): E2M1 codes with one UE4M3 scale per 16 elements
 // along K. Block scales live in 512-byte chunks, one per 128 rows x 64 elements of K; chunk
@@ -83,6 +100,11 @@ struct Nvfp4PrologueArgs {
   const uint8_t* bits_table;
   int32_t bits_index;
   uint32_t* status;
+  // gating (see gated_out): kGateNvfp4 makes the whole launch step aside unless
+  // gate_table[gate_index] is 0
+  int32_t gate;
+  const uint8_t* gate_table;
+  int32_t gate_index;
 };
 cudaError_t launch_prologue_nvfp4(const Nvfp4PrologueArgs& a, cudaStream_t stream);
 
@@ -128,6 +150,7 @@ struct GemmArgs {
   uint32_t* status;
   uint64_t wait_limit_ns;
   int32_t premasked;       // 1: the weight operand already holds mask(w) for this bit width
+  int32_t gate;            // kGateNone, kGateInt8 or kGateNvfp4 (see gated_out), on bits_table[bits_index]
 };
 cudaError_t launch_masked_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const CUtensorMap& tmap_y,
                                const GemmArgs& g, OutKind out, int num_sms, cudaStream_t stream);
