@@ -316,13 +316,32 @@ def time_dmpq(T, torch, ctx, wl, xs, ys, stream, reps: int = 20):
     return {"us": us, "gbs": 4.0 * M * D_in / (us * 1e-6) / 1e9, "shape": [M, D_in], "gamma": float(g.item())}
 
 
+# threshold of the on-device predictor of dmpq_online workloads, set once per run
+DMPQ_TAU = {}
+
+
+def dmpq_block(T, ctx, wl, xs, b, step, stream, gamma_out=None):
+    """The predictor for block b at `step`: its relative L1 change between its input and the next
+    block's input (the last block: its own input against the first block's) picks INT8 (8 bits)
+    or NVFP4 for all its linears, on the device."""
+    per = len(wl.block_layers)
+    K = wl.block_layers[0][1]
+    x_in = xs[b * per]
+    x_out = xs[((b + 1) % wl.blocks) * per]
+    T.tasq_dmpq_update(ctx, x_in, K, x_out, K, wl.tokens, K, [b * per + j for j in range(per)], step,
+                       DMPQ_TAU.get(wl.name, 0.0), 8, T.TASQ_NVFP4, gamma_out, stream)
+
+
 def run_step(T, ctx, wl, xs, ys, step, stream):
     """Every linear of every block once. Linears that read the same input (q, k, v of SDXL) run
-    as one group: one prologue, one GEMM each."""
+    as one group: one prologue, one GEMM each. dmpq_online workloads run the predictor before
+    each block."""
     M = wl.tokens
     per = len(wl.block_layers)
     plan = wl.forward_plan()
     for b in range(wl.blocks):
+        if wl.dmpq_online:
+            dmpq_block(T, ctx, wl, xs, b, step, stream)
         for group in plan:
             l0 = b * per + group[0]
             _, K, N = wl.block_layers[group[0]]
@@ -377,6 +396,8 @@ def run_step_io(T, ctx, wl, xs, ys, step, stream, x_first, y_last):
     per = len(wl.block_layers)
     plan = wl.forward_plan()
     for b in range(wl.blocks):
+        if wl.dmpq_online:
+            dmpq_block(T, ctx, wl, xs, b, step, stream)
         for group in plan:
             l0 = b * per + group[0]
             _, K, N = wl.block_layers[group[0]]
@@ -391,7 +412,11 @@ def run_step_io(T, ctx, wl, xs, ys, step, stream, x_first, y_last):
 
 
 def launches_per_step(wl) -> int:
-    """Kernels one step launches: a prologue per input, a GEMM per linear."""
+    """Kernels one step launches: a prologue per input, a GEMM per linear; with the on-device
+    predictor, one predictor launch per block and both formats' prologue and GEMM per linear
+    (the two of the format not chosen return at once)."""
+    if wl.dmpq_online:
+        return wl.blocks * (1 + 4 * len(wl.block_layers))
     return wl.blocks * (len(wl.forward_plan()) + len(wl.block_layers))
 
 
@@ -596,6 +621,13 @@ def main(argv=None):
                                  args.prologue_mode)
     stream = torch.cuda.current_stream()
     L = wl.num_layers
+    if wl.dmpq_online:
+        # the predictor's threshold: the median of the blocks' relative L1 change, measured once
+        gam = torch.zeros((wl.blocks,), dtype=torch.float64, device=device)
+        for b in range(wl.blocks):
+            dmpq_block(T, ctx, wl, xs, b, 0, stream, gam[b:b + 1])
+        torch.cuda.synchronize()
+        DMPQ_TAU[wl.name] = float(gam.median().item())
 
     for i in range(args.warmup):
         run_step(T, ctx, wl, xs, ys, i % wl.steps, stream)
@@ -655,6 +687,8 @@ def main(argv=None):
     trace = T.tasq_trace_read(ctx)
     T.tasq_trace_enable(ctx, 0)
     status = T.tasq_get_device_status(ctx)
+    # the widths the on-device predictor chose (the last visit of every step)
+    device_table = T.tasq_get_schedule(ctx) if wl.dmpq_online else None
 
     # ---- end to end through the public API: pinned host input in, host result out, per step
     e2e = None
@@ -732,7 +766,7 @@ def main(argv=None):
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl)
 
-    sched = workloads.schedule(wl)
+    sched = device_table if device_table is not None else workloads.schedule(wl)
     used = sched[:, [i % wl.steps for i in range(args.steps)]].astype(np.float64)
     nvfp4 = used == 0
     # weight bits, an NVFP4 step counted as 4; BitOPs model: weight bits x activation bits against

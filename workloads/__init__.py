@@ -55,6 +55,8 @@ class Workload:
     shared_input: Tuple[Tuple[int, ...], ...] = ()
     # relative_l1 schedules: the width of the stable blocks (0 = the NVFP4 step)
     stable_bits: int = 4
+    # the on-device predictor picks every block's format at every step (INT8 8 bits or NVFP4)
+    dmpq_online: bool = False
 
     def forward_plan(self) -> List[Tuple[int, ...]]:
         """The block's linears in order, as tuples of block-layer indices sharing one input."""
@@ -118,6 +120,13 @@ WORKLOADS = {
         name="cogvideox_nvfp4", tokens=13 * 30 * 45 + 226,
         block_layers=(("qkv", 3072, 9216), ("proj", 3072, 3072), ("fc1", 3072, 12288), ("fc2", 12288, 3072)),
         blocks=42, steps=50, hadamard_n=64, schedule_kind="relative_l1", stable_bits=0),
+    # the same split decided on the device each step by the DMPQ predictor (the whole
+    # 6Bit-Diffusion loop): block b's relative L1 change is taken between its input and the next
+    # block's input, the threshold is the median over the blocks of the first step
+    "cogvideox_dmpq": Workload(
+        name="cogvideox_dmpq", tokens=13 * 30 * 45 + 226,
+        block_layers=(("qkv", 3072, 9216), ("proj", 3072, 3072), ("fc1", 3072, 12288), ("fc2", 12288, 3072)),
+        blocks=42, steps=50, hadamard_n=64, schedule_kind="relative_l1", stable_bits=0, dmpq_online=True),
 }
 
 # order of the INT8 workloads as the task lists them (cogvideox_nvfp4 is the NVFP4 variant)
