@@ -66,6 +66,8 @@ def parse_args(argv=None):
                    help="LSB mask: 0 automatic, 1 inside the GEMM on every tile, 2 once ahead in the prologue launch")
     p.add_argument("--bitplanes", default=None,
                    help="workload:layer -- time the bit-plane formulation against the masked dense GEMM")
+    p.add_argument("--nvfp4", action="store_true",
+                   help="with --gemm-shape: time the block-scaled NVFP4 GEMM instead of the INT8 one")
     p.add_argument("--gemm-shape", default=None,
                    help="M,N,K: time the GEMM alone on given codes (one JSON line) and exit")
     p.add_argument("--graph", action="store_true",
@@ -464,20 +466,33 @@ def gemm_shape(args):
     s = torch.cuda.current_stream()
     ctx = T.tasq_linear_create([(N, K, w, s_w)], 1, 64, M, T.TASQ_OUT_F16, s)
     T.tasq_debug_set_gemm_mode(ctx, args.gemm_mode)
+    if args.nvfp4:
+        # random E2M1 code bytes and finite UE4M3 block scales (0x30..0x3F: 0.5 .. 1.875)
+        codes = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        sf = torch.randint(0x30, 0x40, (T.tasq_nvfp4_scale_bytes(M, K),), dtype=torch.uint8, device=dev,
+                           generator=g)
+
+        def call():
+            T.tasq_debug_gemm_nvfp4(ctx, codes, sf, s_x, M, 0, y, N, T.TASQ_OUT_F16, s)
+    else:
+        def call():
+            T.tasq_debug_gemm(ctx, q, s_x, M, 0, 0, y, N, T.TASQ_OUT_F16, s)
     for _ in range(3):
-        T.tasq_debug_gemm(ctx, q, s_x, M, 0, 0, y, N, T.TASQ_OUT_F16, s)
+        call()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(s)
     for _ in range(args.reps):
-        T.tasq_debug_gemm(ctx, q, s_x, M, 0, 0, y, N, T.TASQ_OUT_F16, s)
+        call()
     e1.record(s)
     torch.cuda.synchronize()
     us = 1e3 * e0.elapsed_time(e1) / args.reps
     peaks, _ = load_peaks()
     tops = 2.0 * M * N * K / (us * 1e-6) / 1e12
-    print(json.dumps({"gemm_shape": [M, N, K], "gemm_mode": args.gemm_mode, "us": us, "tops": tops,
+    # the NVFP4 hook converts the layer's weights (one prologue launch) before each GEMM
+    print(json.dumps({"gemm_shape": [M, N, K], "nvfp4": bool(args.nvfp4), "gemm_mode": args.gemm_mode, "us": us,
+                      "includes_weight_conversion": bool(args.nvfp4), "tops": tops,
                       "frac_int8_burst": tops / (peaks["bf16_tflops"] * INT8_OVER_BF16),
                       "device_status": T.tasq_get_device_status(ctx)}), flush=True)
     return 0

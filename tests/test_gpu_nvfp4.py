@@ -156,7 +156,8 @@ def _terms_bound(ca, sa, cw, sw, Kp):
 
 @pytest.mark.parametrize("M,N,K,n", [(1, 8, 64, 64), (130, 200, 1152, 64), (300, 520, 320, 64),
                                      (257, 1152, 4608, 64), (64, 2000, 2240, 128), (513, 384, 12288, 64)])
-def test_nvfp4_gemm_accumulators(T, M, N, K, n):
+@pytest.mark.parametrize("mode", [1, 2], ids=["one_cta", "cta_pair"])
+def test_nvfp4_gemm_accumulators(T, M, N, K, n, mode):
     rng = np.random.default_rng(M * 3 + N + K)
     Kp = oracle.padded_k(K, n)
     w = rng.integers(-127, 128, size=(N, Kp)).astype(np.int8)
@@ -164,6 +165,7 @@ def test_nvfp4_gemm_accumulators(T, M, N, K, n):
     ca, sa, sx, _ = oracle.nvfp4_prologue(x, n)
     cw, sw = oracle.nvfp4_quantize_weights(w)
     ctx = _ctx(T, [(N, K, w, np.ones(N, np.float32))], 1, n, M)
+    T.tasq_debug_set_gemm_mode(ctx, mode)
     codes = _dev(oracle.pack_nibbles(ca))
     sf = _dev(chunk_scales(sa, Kp))
     sxd = _dev(sx.astype(np.float32))
@@ -182,7 +184,8 @@ def test_nvfp4_gemm_accumulators(T, M, N, K, n):
 # ----------------------------------------------------------------------------- whole forward
 @pytest.mark.parametrize("n,K,N,M", [(64, 1152, 1152, 256), (64, 1152, 3456, 300), (128, 2240, 6720, 130),
                                      (64, 4608, 1152, 77), (64, 64, 8, 1)])
-def test_nvfp4_forward_matches_oracle(T, n, K, N, M):
+@pytest.mark.parametrize("mode", [0, 1, 2], ids=["auto", "one_cta", "cta_pair"])
+def test_nvfp4_forward_matches_oracle(T, n, K, N, M, mode):
     rng = np.random.default_rng(n + K + N + M)
     Kp = oracle.padded_k(K, n)
     x = _acts(rng, M, K)
@@ -190,6 +193,7 @@ def test_nvfp4_forward_matches_oracle(T, n, K, N, M):
     s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
     bits = [8, T.TASQ_NVFP4, 5, T.TASQ_NVFP4]
     ctx = _ctx(T, [(N, K, w, s_w)], len(bits), n, M + 3)
+    T.tasq_debug_set_gemm_mode(ctx, mode)
     T.tasq_set_schedule(ctx, np.array([bits], np.uint8), _stream())
     xd = _dev(x)
     ldy = N + (8 - N % 8) % 8 + 8

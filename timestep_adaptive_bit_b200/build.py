@@ -11,7 +11,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libtasq.so")
-SOURCES = ("tasq_api.cu", "prologue.cu", "masked_gemm.cu", "masked_gemm_pair.cu", "gemm_nvfp4.cu", "noalloc.cu",
+SOURCES = ("tasq_api.cu", "prologue.cu", "masked_gemm.cu", "masked_gemm_pair.cu", "gemm_nvfp4.cu",
+           "gemm_nvfp4_pair.cu", "noalloc.cu",
            "dmpq.cu")
 
 

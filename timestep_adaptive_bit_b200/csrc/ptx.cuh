@@ -350,6 +350,26 @@ __device__ __forceinline__ void mma_i8_ss_pair(uint32_t d_tmem, uint64_t a_desc,
       : "memory");
 }
 
+// Block-scaled NVFP4 MMA over a CTA pair (kind::mxf4nvf4, scale_vec::4X, K = 64): each CTA
+// supplies half of A's rows and half of B's rows from the same shared-memory offsets; each CTA's
+// TMEM holds the scales of its own A rows at sfa_tmem and the scales of all N rows of B at
+// sfb_tmem. Issued by the pair's first CTA only.
+__device__ __forceinline__ void mma_nvfp4_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// tmem_cp_32x128b_warpx4 for a CTA pair: every CTA's 512-byte block at the descriptor's
+// shared-memory offset goes into its own TMEM at taddr. Issued by the pair's first CTA only.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrive once on the barrier at cluster address `bar` when every pair MMA this thread issued so
 // far has completed.
 __device__ __forceinline__ void mma_commit_pair(uint32_t bar) {

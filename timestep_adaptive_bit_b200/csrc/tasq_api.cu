@@ -344,11 +344,15 @@ tasq_status run_gemm_nvfp4(tasq_ctx* c, int32_t layer, int32_t step, const uint8
                            cudaStream_t s, int32_t gate = tasq::kGateNone) {
   const LayerInfo& L = c->layers[layer];
   const int64_t kp4 = tasq::nvfp4_kp4(L.Kp);
+  const bool pair = c->gemm_mode == 2 || (c->gemm_mode == 0 && tasq::nvfp4_use_pair(M, L.N, c->num_sms));
+  const int tile_tok = pair ? tasq::kGemmNvfp4PairTok : 128;
+  const int tile_ch = pair ? 256 : 128;
   CUtensorMap tw, tx, ty;
   tasq_status st = make_tmap_u8(&tw, nvfp4_w_codes(c, slot), static_cast<uint64_t>(L.Kp / 2),
                                 static_cast<uint64_t>(L.N), 128, 128);
   if (st == TASQ_OK)
-    st = make_tmap_u8(&tx, codes, static_cast<uint64_t>(L.Kp / 2), static_cast<uint64_t>(M), 128, 128);
+    st = make_tmap_u8(&tx, codes, static_cast<uint64_t>(L.Kp / 2), static_cast<uint64_t>(M), 128,
+                      static_cast<uint32_t>(pair ? tile_tok / 2 : tile_tok));
   if (st != TASQ_OK) return st;
   const CUtensorMapDataType dt = out == tasq::OutKind::S32    ? CU_TENSOR_MAP_DATA_TYPE_INT32
                                  : out == tasq::OutKind::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -360,8 +364,8 @@ tasq_status run_gemm_nvfp4(tasq_ctx* c, int32_t layer, int32_t step, const uint8
   g.M = static_cast<int32_t>(M);
   g.N = L.N;
   g.num_kb = static_cast<int32_t>(kp4 / 256);
-  g.num_m_tiles = static_cast<int32_t>((M + 127) / 128);
-  g.num_n_tiles = (L.N + 127) / 128;
+  g.num_m_tiles = static_cast<int32_t>((M + tile_tok - 1) / tile_tok);
+  g.num_n_tiles = (L.N + tile_ch - 1) / tile_ch;
   g.bits_table = step < 0 ? nullptr : c->d_bits;
   g.bits_index = layer * c->num_steps + (step < 0 ? 0 : step);
   g.s_x = sx;
@@ -375,8 +379,9 @@ tasq_status run_gemm_nvfp4(tasq_ctx* c, int32_t layer, int32_t step, const uint8
   f.w_sf = nvfp4_w_sf(c, layer, slot);
   f.x_sf = sf;
   f.sf_chunks = static_cast<int32_t>(kp4 / 64);
-  cudaError_t e = tasq::launch_gemm_nvfp4(tw, tx, ty, g, f, out, c->num_sms, s);
-  if (e != cudaSuccess) return fail_cuda(e, "NVFP4 GEMM launch");
+  cudaError_t e = pair ? tasq::launch_gemm_nvfp4_pair(tw, tx, ty, g, f, out, c->num_sms, s)
+                       : tasq::launch_gemm_nvfp4(tw, tx, ty, g, f, out, c->num_sms, s);
+  if (e != cudaSuccess) return fail_cuda(e, pair ? "NVFP4 pair GEMM launch" : "NVFP4 GEMM launch");
   return TASQ_OK;
 }
 
@@ -402,6 +407,18 @@ bool gemm_use_pair(int64_t M, int64_t N, int num_sms) {
   const int64_t w1 = (t1 + slots1 - 1) / slots1;
   const int64_t w2 = (t2 + slots2 - 1) / slots2;
   return w2 < w1 || (w2 == w1 && w1 >= 4);
+}
+
+// The NVFP4 kernels by estimated time, waves x time per tile: a pair tile (256 x 192 on two SMs)
+// holds 1.5x the MACs per SM of a one-CTA tile (128 x 128) and runs them 1.37x faster (CogVideoX
+// qkv, 17776 x 3072 -> 9216, CUDA events), so it takes about 1.1x as long.
+bool nvfp4_use_pair(int64_t M, int64_t N, int num_sms) {
+  const int64_t t1 = ((M + 127) / 128) * ((N + 127) / 128);
+  const int64_t t2 = ((M + kGemmNvfp4PairTok - 1) / kGemmNvfp4PairTok) * ((N + 255) / 256);
+  const int64_t slots1 = num_sms, slots2 = num_sms / 2;
+  const int64_t w1 = (t1 + slots1 - 1) / slots1;
+  const int64_t w2 = (t2 + slots2 - 1) / slots2;
+  return 110 * w2 <= 100 * w1;
 }
 
 }  // namespace tasq

@@ -168,6 +168,18 @@ cudaError_t launch_gemm_nvfp4(const CUtensorMap& tmap_w, const CUtensorMap& tmap
                               const GemmArgs& g, const Nvfp4GemmArgs& f, OutKind out, int num_sms,
                               cudaStream_t stream);
 
+// The NVFP4 GEMM over CTA pairs (tcgen05 cta_group::2): tiles of 256 channels x 192 tokens, each
+// CTA holding 128 weight rows and 96 token rows per stage (tensor-map boxes of 128 x 128 and
+// 96 x 128 bytes), g.num_m_tiles = ceil(M / 192), g.num_n_tiles = ceil(N / 256); the scales in
+// the same chunked layout as launch_gemm_nvfp4.
+constexpr int kGemmNvfp4PairTok = 192;   // tokens per NVFP4 pair tile
+cudaError_t launch_gemm_nvfp4_pair(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const CUtensorMap& tmap_y,
+                                   const GemmArgs& g, const Nvfp4GemmArgs& f, OutKind out, int num_sms,
+                                   cudaStream_t stream);
+// Whether the automatic choice runs an NVFP4 GEMM of M tokens and N channels on CTA pairs
+// (defined in tasq_api.cu).
+bool nvfp4_use_pair(int64_t M, int64_t N, int num_sms);
+
 // The same GEMM over CTA pairs (tcgen05 cta_group::2): tiles of 256 channels x 256 tokens, each
 // CTA holding 128 rows of each operand (tensor-map boxes of 128 x 128 bytes for both).
 cudaError_t launch_masked_gemm_pair(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const CUtensorMap& tmap_y,
