@@ -217,6 +217,33 @@ def test_nvfp4_forward_matches_oracle(T, n, K, N, M, mode):
     assert T.tasq_get_device_status(ctx) == 0
 
 
+@pytest.mark.parametrize("mode", [1, 2], ids=["one_cta", "cta_pair"])
+def test_nvfp4_forward_bf16_output(T, mode):
+    """BF16 outputs of an NVFP4 step: the FP32 bound of the accumulators carried through the
+    scales, plus the BF16 rounding (8 significant bits: half an ulp is at most 2^-8 of |y|)."""
+    rng = np.random.default_rng(77 + mode)
+    n, K, N, M = 64, 1152, 1000, 389     # odd and even 192-token tiles, a ragged channel tile
+    Kp = oracle.padded_k(K, n)
+    x = _acts(rng, M, K)
+    w = rng.integers(-127, 128, size=(N, Kp)).astype(np.int8)
+    s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+    ctx = T.tasq_linear_create([(N, K, w, s_w)], 1, n, M, T.TASQ_OUT_BF16, _stream())
+    T.tasq_debug_set_gemm_mode(ctx, mode)
+    T.tasq_set_schedule(ctx, np.array([[T.TASQ_NVFP4]], np.uint8), _stream())
+    ldy = 1008
+    y = torch.full((M + 1, ldy), float("nan"), dtype=torch.bfloat16, device="cuda")
+    T.tasq_linear_forward(ctx, _dev(x), M, K, 0, 0, y, ldy, _stream())
+    torch.cuda.synchronize()
+    got = y.float().cpu().numpy()
+    assert np.all(np.isnan(got[M:])) and np.all(np.isnan(got[:M, N:])), "write outside [M, N]"
+    got = got[:M, :N].astype(np.float64)
+    r4 = oracle.nvfp4_linear(x, w, s_w, n)
+    bound = _terms_bound(r4["ca"], r4["sa"], r4["cw"], r4["sw"], Kp) * r4["s_x"][:, None] * s_w[None, :]
+    tol = bound * 1.0001 + np.abs(r4["y"]) * (2.0 ** -8 + 2.0 ** -21) + 2.0 ** -24
+    assert np.all(np.abs(got - r4["y"]) <= tol)
+    assert T.tasq_get_device_status(ctx) == 0
+
+
 def test_nvfp4_and_int8_layers_interleave(T):
     """Two layers, NVFP4 and INT8 steps back to back on one stream: each forward reads its own
     weights, the NVFP4 weights never leak into the INT8 path (they share the masked-weight slot)."""
