@@ -67,7 +67,8 @@ def parse_args(argv=None):
     p.add_argument("--bitplanes", default=None,
                    help="workload:layer -- time the bit-plane formulation against the masked dense GEMM")
     p.add_argument("--nvfp4", action="store_true",
-                   help="with --gemm-shape: time the block-scaled NVFP4 GEMM instead of the INT8 one")
+                   help="with --gemm-shape: time the block-scaled NVFP4 GEMM instead of the INT8 one; "
+                        "with --sweep-bits: add an NVFP4 step (reported as width 0)")
     p.add_argument("--gemm-shape", default=None,
                    help="M,N,K: time the GEMM alone on given codes (one JSON line) and exit")
     p.add_argument("--graph", action="store_true",
@@ -570,11 +571,13 @@ def sweep_bits(args):
     dev = torch.device("cuda:0")
     w, s_w = workloads.weights_torch(wl, j, dev)
     s = torch.cuda.current_stream()
-    ctx = T.tasq_linear_create([(N, K, w, s_w)], 8, wl.hadamard_n, M, T.TASQ_OUT_F16, s)
+    # bit widths 8 .. 1, then (with --nvfp4) one NVFP4 step, reported under "0"
+    widths = [8, 7, 6, 5, 4, 3, 2, 1] + ([0] if args.nvfp4 else [])
+    ctx = T.tasq_linear_create([(N, K, w, s_w)], len(widths), wl.hadamard_n, M, T.TASQ_OUT_F16, s)
     T.tasq_debug_set_gemm_mode(ctx, args.gemm_mode)
     T.tasq_debug_set_mask_mode(ctx, args.mask_mode)
     T.tasq_debug_set_prologue_mode(ctx, args.prologue_mode)
-    T.tasq_set_schedule(ctx, np.array([[8, 7, 6, 5, 4, 3, 2, 1]], np.uint8), s)
+    T.tasq_set_schedule(ctx, np.array([widths], np.uint8), s)
     # several input buffers so consecutive launches do not find their activations in L2
     nbuf = max(2, int(math.ceil(3 * 126e6 / (M * K * 2))))
     xs = [workloads.activations_torch(wl, j, dev, seed=b) for b in range(nbuf)]
@@ -583,7 +586,7 @@ def sweep_bits(args):
     out = {"sweep": f"{name}:{wl.block_layers[j][0]}", "M": M, "K": K, "N": N, "reps": args.reps,
            "gemm_mode": args.gemm_mode, "mask_mode": args.mask_mode, "prologue_mode": args.prologue_mode,
            "bits": {}}
-    for step in range(8):
+    for step, width in enumerate(widths):
         for r in range(3):
             T.tasq_linear_forward(ctx, xs[r % nbuf], M, K, 0, step, y, N, s)
         torch.cuda.synchronize()
@@ -593,7 +596,7 @@ def sweep_bits(args):
         tr = T.tasq_trace_read(ctx)
         g_tops = tr["gemm_ops"] / (tr["gemm_ms"] / 1e3) / 1e12
         p_gbs = tr["prologue_bytes"] / (tr["prologue_ms"] / 1e3) / 1e9
-        out["bits"][8 - step] = {"gemm_us": 1e3 * tr["gemm_ms"] / args.reps, "gemm_tops": g_tops,
+        out["bits"][width] = {"gemm_us": 1e3 * tr["gemm_ms"] / args.reps, "gemm_tops": g_tops,
                                  "gemm_frac_int8_burst": g_tops / (peaks["bf16_tflops"] * INT8_OVER_BF16),
                                  "prologue_us": 1e3 * tr["prologue_ms"] / args.reps, "prologue_gbs": p_gbs,
                                  "prologue_frac_hbm": p_gbs / peaks["hbm_gbs"],

@@ -68,7 +68,8 @@ def _ctx(T, layers, steps, n, max_tokens):
 
 # ----------------------------------------------------------------------------- prologue
 @pytest.mark.parametrize("n,K,M", [(64, 64, 1), (64, 1152, 257), (128, 2240, 130), (64, 4608, 300),
-                                   (64, 12288, 33), (128, 5600, 64), (64, 1280, 4097), (64, 96, 3)])
+                                   (64, 12288, 33), (128, 10240, 40), (128, 5600, 64), (64, 1280, 4097),
+                                   (64, 96, 3)])
 def test_nvfp4_prologue_matches_oracle(T, n, K, M):
     rng = np.random.default_rng(K + 7 * M)
     x = _acts(rng, M, K)

@@ -44,6 +44,7 @@ namespace {
 constexpr int kMaxRowsPerCta = 64;
 constexpr int kMaxThreads = 512;
 constexpr int kSmallThreads = 288;   // CTAs up to this size get 56 registers: 4 CTAs per SM
+constexpr int kMidThreads = 384;     // NVFP4 prologue: CTAs up to this size get 56 registers, 3 per SM
 
 __device__ __forceinline__ uint4 ld_16B(const void* p) {
   uint4 v;
@@ -362,9 +363,10 @@ __device__ __forceinline__ int64_t nvfp4_sf_offset(int64_t r, int64_t j, int64_t
   return ((r >> 7) * chunks_per_group + (j >> 2)) * kNvfp4ChunkBytes + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (j & 3);
 }
 
-// NVFP4 codes and scale of the 16 INT8 weights w[0..15] (one block of one output channel).
-__device__ __forceinline__ void nvfp4_weight_block(const int8_t* w, uint8_t* codes, uint8_t* sf_byte) {
-  const uint4 q = *reinterpret_cast<const uint4*>(w);
+// NVFP4 codes and scale of 16 INT8 weights (one block of one output channel), given as the four
+// 32-bit words that hold them: 8 bytes of E2M1 codes (lower-indexed element in the low nibble)
+// and the UE4M3 scale byte.
+__device__ __forceinline__ uint32_t nvfp4_weight_block(const uint4 q, uint2* codes) {
   const uint32_t words[4] = {q.x, q.y, q.z, q.w};
   float f[16];
   int m = 0;
@@ -383,29 +385,45 @@ __device__ __forceinline__ void nvfp4_weight_block(const int8_t* w, uint8_t* cod
     t0[i] = __fmul_rn(f[i], r);
     t1[i] = __fmul_rn(f[8 + i], r);
   }
-  uint2 out = make_uint2(e2m1_x8(t0), e2m1_x8(t1));
-  if (d == 0.0f) out = make_uint2(0u, 0u);
-  *reinterpret_cast<uint2*>(codes) = out;
-  *sf_byte = static_cast<uint8_t>(sc);
+  *codes = d == 0.0f ? make_uint2(0u, 0u) : make_uint2(e2m1_x8(t0), e2m1_x8(t1));
+  return sc;
 }
 
-// Weight conversion of CTA `cta` of `num_ctas`: one thread per 16-block, then zero scales for
-// the blocks between Kp and Kp4, so that the GEMM's last stage multiplies zero codes by zero.
-__device__ __forceinline__ void nvfp4_weight_pass(const Nvfp4PrologueArgs& a, int64_t cta, int64_t num_ctas) {
+// Weight conversion of CTA `cta` of `num_ctas`. One thread per four consecutive 16-blocks of a
+// row: 64 INT8 weights in (four independent 16-byte loads), 32 bytes of codes and one 32-bit word
+// of scales out (the four blocks' scales are adjacent bytes of the chunked layout). Quads past Kp
+// (Kp is a multiple of 64, so a quad is wholly inside or outside) get zero scales, so that the
+// GEMM's last stage multiplies zero codes by zero.
+__device__ __forceinline__ void nvfp4_weight_pass(const Nvfp4PrologueArgs& a, int cta, int num_ctas) {
   // the previous GEMM may still read the converted weights: wait for it
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (cta == 0 && threadIdx.x == 0 && a.bits_table != nullptr && a.bits_table[a.bits_index] != 0)
     atomicOr(a.status, TASQ_DEVICE_BAD_BITS);
-  const int64_t nb = a.Kp / kNvfp4Block;
-  const int64_t nb4 = nvfp4_kp4(a.Kp) / kNvfp4Block;
-  const int64_t chunks = nb4 / 4;
-  const int64_t stride = num_ctas * blockDim.x;
-  for (int64_t i = cta * blockDim.x + threadIdx.x; i < static_cast<int64_t>(a.N) * nb4; i += stride) {
-    const int64_t row = i / nb4, j = i - row * nb4;
-    uint8_t* sf = a.w_sf + nvfp4_sf_offset(row, j, chunks);
-    if (j < nb) nvfp4_weight_block(a.w + row * a.Kp + 16 * j, a.w_codes + row * (a.Kp / 2) + 8 * j, sf);
-    else *sf = 0;
+  const int nb = a.Kp / kNvfp4Block;
+  const int quads = static_cast<int>(nvfp4_kp4(a.Kp) / 64);   // per row; = scale chunks per row group
+  const int total = a.N * quads;
+  const int stride = num_ctas * static_cast<int>(blockDim.x);
+  for (int qd = cta * static_cast<int>(blockDim.x) + static_cast<int>(threadIdx.x); qd < total; qd += stride) {
+    const int row = qd / quads;
+    const int j0 = 4 * (qd - row * quads);
+    uint32_t* sf = reinterpret_cast<uint32_t*>(a.w_sf + nvfp4_sf_offset(row, j0, quads));
+    if (j0 >= nb) {
+      *sf = 0u;
+      continue;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(a.w + static_cast<int64_t>(row) * a.Kp + 16 * j0);
+    uint4 q[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) q[b] = __ldg(src + b);
+    uint2 c[4];
+    uint32_t scales = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) scales |= nvfp4_weight_block(q[b], &c[b]) << (8 * b);
+    uint4* dst = reinterpret_cast<uint4*>(a.w_codes + static_cast<int64_t>(row) * (a.Kp / 2) + 8 * j0);
+    dst[0] = make_uint4(c[0].x, c[0].y, c[1].x, c[1].y);
+    dst[1] = make_uint4(c[2].x, c[2].y, c[3].x, c[3].y);
+    *sf = scales;
   }
 }
 
@@ -413,15 +431,19 @@ template <int LANES, int MAXT, int MINB>
 __global__ void __launch_bounds__(MAXT, MINB)
     prologue_nvfp4_kernel(const Nvfp4PrologueArgs a, const int rows_per_cta, const int row_ctas) {
   if (gated_out(a.gate, a.gate_table, a.gate_index)) return;
-  if (static_cast<int>(blockIdx.x) >= row_ctas) {
-    nvfp4_weight_pass(a, blockIdx.x - row_ctas, gridDim.x - row_ctas);
+  // CTAs [0, weight_ctas) convert the weights (each loops over several quads, so they start
+  // first), the rest quantize activation rows
+  const int weight_ctas = static_cast<int>(gridDim.x) - row_ctas;
+  if (static_cast<int>(blockIdx.x) < weight_ctas) {
+    nvfp4_weight_pass(a, blockIdx.x, weight_ctas);
     return;
   }
+  const int row_block = static_cast<int>(blockIdx.x) - weight_ctas;
   const int L = a.Kp >> 5;
   const int tid = threadIdx.x;
   const int r_local = tid / L;
   const int seg = tid - r_local * L;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + r_local;
+  const int64_t row = static_cast<int64_t>(row_block) * rows_per_cta + r_local;
   const bool active = r_local < rows_per_cta && row < a.M;
 
   // x may be the previous kernel's output, and the previous GEMM may still read the codes
@@ -797,18 +819,23 @@ cudaError_t launch_prologue_nvfp4(const Nvfp4PrologueArgs& a, cudaStream_t strea
     return cudaErrorInvalidValue;
   const int L = a.Kp / 32;
   if (L > kMaxThreads) return cudaErrorInvalidValue;
+  // rows of up to 288 threads run in CTAs of at most 288 threads, four per SM; rows of up to
+  // 384 threads (K = 12288) one per CTA, three per SM; longer rows take the 512-thread instance
   const bool small = L <= kSmallThreads;
+  const bool mid = !small && L <= kMidThreads;
   int R = 1, threads = 256;
   int64_t row_ctas = 0;
   if (a.M > 0) {
-    R = pick_rows(L, small ? kSmallThreads : kMaxThreads);
+    R = pick_rows(L, small ? kSmallThreads : mid ? kMidThreads : kMaxThreads);
     threads = ((R * L + 31) / 32) * 32;
     row_ctas = (a.M + R - 1) / R;
   }
   int64_t weight_ctas = 0;
   if (weights) {
-    const int64_t blocks = static_cast<int64_t>(a.N) * (nvfp4_kp4(a.Kp) / kNvfp4Block);
-    weight_ctas = (blocks + threads - 1) / threads;
+    // one thread per four 16-blocks of a row
+    const int64_t quads = static_cast<int64_t>(a.N) * (nvfp4_kp4(a.Kp) / 64);
+    if (quads > 0x7fffffffLL) return cudaErrorInvalidValue;
+    weight_ctas = (quads + threads - 1) / threads;
     if (weight_ctas > kMaxWeightCtas) weight_ctas = kMaxWeightCtas;
   }
   const int64_t grid = row_ctas + weight_ctas;
@@ -826,6 +853,10 @@ cudaError_t launch_prologue_nvfp4(const Nvfp4PrologueArgs& a, cudaStream_t strea
   if (small) {
     if (a.n == 64) return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<2, kSmallThreads, 4>, a, R, rc);
     return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<4, kSmallThreads, 4>, a, R, rc);
+  }
+  if (mid) {
+    if (a.n == 64) return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<2, kMidThreads, 3>, a, R, rc);
+    return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<4, kMidThreads, 3>, a, R, rc);
   }
   if (a.n == 64) return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<2, kMaxThreads, 1>, a, R, rc);
   return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<4, kMaxThreads, 1>, a, R, rc);
