@@ -689,7 +689,11 @@ def main(argv=None):
     # ---- per-kernel durations: a separate pass of the same steps with CUDA events around every
     # kernel. Events between the kernels break their programmatic-launch overlap (about 18 % on
     # the PixArt-Sigma step), so the headline above is timed without them.
+    # whole cycles of the schedule where the timed steps cover one, so that every step's widths
+    # weigh as much as in the timed steps
     trace_steps = max(1, min(args.steps, 40))
+    if args.steps >= wl.steps:
+        trace_steps = max(wl.steps, (trace_steps // wl.steps) * wl.steps)
     T.tasq_trace_enable(ctx, trace_steps * L)
     if dist is not None:
         dist.barrier()
@@ -716,7 +720,8 @@ def main(argv=None):
         x_host = torch.empty((wl.tokens, first_K), dtype=torch.float16, pin_memory=True)
         x_host.copy_(xs[0].cpu())
         y_host = torch.empty((wl.tokens, last_N), dtype=ys[last_N].dtype, pin_memory=True)
-        e_steps = max(1, min(args.steps, 50))
+        # the same steps, in the same order, as the timed loop (the schedule's widths vary by step)
+        e_steps = max(1, args.steps)
         # every step copies its input in from pinned host memory and its result out; the copies run
         # on their own stream into double buffers, so step i's result leaves and step i + 1's input
         # arrives while the GPU computes
