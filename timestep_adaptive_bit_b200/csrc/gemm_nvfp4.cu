@@ -21,6 +21,8 @@
 //   warps 0-7  the INT8 kernels' epilogue, reading FP32 accumulators.
 // Every wait is bounded; a wait that runs out records a status bit, raises the CTA's abort flag,
 // and every role winds down as in the INT8 kernels.
+#include <mutex>
+
 #include "gemm_common.cuh"
 
 namespace tasq {
@@ -229,15 +231,19 @@ template <int OUT>
 cudaError_t launch_f4(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ty, const GemmArgs& g,
                       const Nvfp4GemmArgs& f, int num_sms, cudaStream_t stream) {
   static bool configured[64] = {false};
+  static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
-    e = cudaFuncSetAttribute(gemm_nvfp4_kernel<OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             PlanF4<OUT>::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!configured[dev]) {
+      e = cudaFuncSetAttribute(gemm_nvfp4_kernel<OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               PlanF4<OUT>::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      configured[dev] = true;
+    }
   }
   const int tiles = g.num_m_tiles * g.num_n_tiles;
   const int grid = tiles < num_sms ? tiles : num_sms;

@@ -47,6 +47,8 @@
 // Every wait is bounded; at the end the two CTAs meet on a pair barrier (bounded) before TMEM is
 // freed, so that no CTA leaves while the other's MMAs may still read its shared memory or write
 // its TMEM.
+#include <mutex>
+
 #include "gemm_common.cuh"
 
 namespace tasq {
@@ -408,37 +410,43 @@ cudaError_t launch_pair_f4(const CUtensorMap& tw, const CUtensorMap& tx, const C
                            const Nvfp4GemmArgs& f, int num_sms, cudaStream_t stream) {
   static bool configured[64] = {false};
   static int max_pairs[64] = {0};
+  static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
-    e = cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             PairPlanF4<OUT>::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    // how many CTA pairs can be resident at once on this device
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
-    cfg.blockDim = dim3(kThreadsP4, 1, 1);
-    cfg.dynamicSmemBytes = PairPlanF4<OUT>::kSmemBytes;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, gemm_nvfp4_pair_kernel<OUT>, &cfg);
-    if (e != cudaSuccess || clusters <= 0) {
-      (void)cudaGetLastError();
-      clusters = num_sms / 2;
+  int resident_pairs = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!configured[dev]) {
+      e = cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               PairPlanF4<OUT>::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      // how many CTA pairs can be resident at once on this device
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+      cfg.blockDim = dim3(kThreadsP4, 1, 1);
+      cfg.dynamicSmemBytes = PairPlanF4<OUT>::kSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      e = cudaOccupancyMaxActiveClusters(&clusters, gemm_nvfp4_pair_kernel<OUT>, &cfg);
+      if (e != cudaSuccess || clusters <= 0) {
+        (void)cudaGetLastError();
+        clusters = num_sms / 2;
+      }
+      max_pairs[dev] = clusters;
+      configured[dev] = true;
     }
-    max_pairs[dev] = clusters;
-    configured[dev] = true;
+    resident_pairs = max_pairs[dev];
   }
   const int tiles = g.num_m_tiles * g.num_n_tiles;
-  const int pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
+  const int pairs = tiles < resident_pairs ? tiles : resident_pairs;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(kThreadsP4, 1, 1);

@@ -34,6 +34,8 @@
 // Every wait is bounded (ptx::wait_bounded); a wait that runs out records a status bit, raises
 // a CTA-wide abort flag, and every role winds down: the producer waits (bounded) for the loads
 // it issued, the MMA thread for its MMAs, then TMEM is freed and the CTA exits.
+#include <mutex>
+
 #include "gemm_common.cuh"
 
 namespace tasq {
@@ -274,15 +276,19 @@ template <int OUT>
 cudaError_t launch_out(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ty, const GemmArgs& g,
                        int num_sms, cudaStream_t stream) {
   static bool configured[64] = {false};
+  static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
-    e = cudaFuncSetAttribute(masked_gemm_kernel<OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Plan<OUT>::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!configured[dev]) {
+      e = cudaFuncSetAttribute(masked_gemm_kernel<OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Plan<OUT>::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      configured[dev] = true;
+    }
   }
   const int tiles = g.num_m_tiles * g.num_n_tiles;
   const int grid = tiles < num_sms ? tiles : num_sms;

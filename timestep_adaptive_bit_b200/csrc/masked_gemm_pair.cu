@@ -24,6 +24,8 @@
 #include <cstdio>
 #include <cstdlib>
 
+#include <mutex>
+
 #include "gemm_common.cuh"
 
 namespace tasq {
@@ -276,40 +278,46 @@ cudaError_t launch_pair_out(const CUtensorMap& tw, const CUtensorMap& tx, const 
                             int num_sms, cudaStream_t stream) {
   static bool configured[64] = {false};
   static int max_pairs[64] = {0};
+  static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
-    e = cudaFuncSetAttribute(masked_gemm_pair_kernel<OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             PairPlan<OUT>::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    // how many CTA pairs can be resident at once on this device
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = PairPlan<OUT>::kSmemBytes;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, masked_gemm_pair_kernel<OUT>, &cfg);
-    if (e != cudaSuccess || clusters <= 0) {
-      (void)cudaGetLastError();
-      clusters = num_sms / 2;
+  int resident_pairs = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!configured[dev]) {
+      e = cudaFuncSetAttribute(masked_gemm_pair_kernel<OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               PairPlan<OUT>::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      // how many CTA pairs can be resident at once on this device
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = PairPlan<OUT>::kSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      e = cudaOccupancyMaxActiveClusters(&clusters, masked_gemm_pair_kernel<OUT>, &cfg);
+      if (e != cudaSuccess || clusters <= 0) {
+        (void)cudaGetLastError();
+        clusters = num_sms / 2;
+      }
+      max_pairs[dev] = clusters;
+      configured[dev] = true;
+      if (std::getenv("TASQ_VERBOSE") != nullptr)
+        std::fprintf(stderr, "tasq: pair GEMM on device %d: %d resident CTA pairs, %d bytes of shared memory\n", dev,
+                     clusters, PairPlan<OUT>::kSmemBytes);
     }
-    max_pairs[dev] = clusters;
-    configured[dev] = true;
-    if (std::getenv("TASQ_VERBOSE") != nullptr)
-      std::fprintf(stderr, "tasq: pair GEMM on device %d: %d resident CTA pairs, %d bytes of shared memory\n", dev,
-                   clusters, PairPlan<OUT>::kSmemBytes);
+    resident_pairs = max_pairs[dev];
   }
   const int tiles = g.num_m_tiles * g.num_n_tiles;
-  const int pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
+  const int pairs = tiles < resident_pairs ? tiles : resident_pairs;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
