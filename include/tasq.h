@@ -291,6 +291,17 @@ tasq_status tasq_debug_set_gemm_mode(tasq_ctx* ctx, int32_t mode);
 tasq_status tasq_gemm_choice(int64_t M, int32_t N, int32_t num_sms, int32_t* pair);
 
 /*
+ * Host-only query (no device, no context), the NVFP4 counterpart of tasq_gemm_choice: whether an
+ * NVFP4 step with the automatic choice runs its block-scaled GEMM of M tokens and N output
+ * channels on CTA pairs (*pair = 1, tiles of 256 channels x 192 tokens) or on one CTA per tile
+ * (*pair = 0, 128 x 128). The pair is taken unless it needs more than 1/1.1 as many waves of
+ * tiles as the one-CTA kernel: a pair tile holds 1.5x the MACs per SM and runs them about 1.37x
+ * faster (6Bit-Diffusion's NVFP4 stable-layer step; see tasq_set_schedule). TASQ_ERR_INVALID_ARG
+ * for a NULL output, M or N <= 0, or num_sms < 2.
+ */
+tasq_status tasq_nvfp4_gemm_choice(int64_t M, int32_t N, int32_t num_sms, int32_t* pair);
+
+/*
  * Test hook: where later forwards (and tasq_debug_gemm / tasq_debug_gemm_s32) apply the step's
  * LSB mask to the weights (TASQ, "LSB masking" of the stored INT8 weights). 0 (default): ahead of
  * the GEMM, in the prologue launch, into a context-owned copy of the layer's weights whenever the

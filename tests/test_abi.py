@@ -138,3 +138,28 @@ def test_gemm_choice_is_host_only(tasq):
         with pytest.raises(tasq.TasqError) as ei:
             tasq.tasq_gemm_choice(*bad)
         assert ei.value.status == tasq.TASQ_ERR_INVALID_ARG
+
+
+def test_nvfp4_gemm_choice_is_host_only(tasq):
+    """The automatic NVFP4 GEMM kernel choice is a host function of (M, N, SM count). On the
+    workloads' shapes it picks the kernel that CUDA-event timings of both NVFP4 kernels on a B200
+    (148 SMs, bench.py --gemm-shape M,N,K --nvfp4 --gemm-mode 1|2) found faster: CTA pairs
+    everywhere except SANA's 2240-channel linears and a 256-token linear, where the two differ by
+    at most 5 %."""
+    faster_on_b200 = {
+        (8192, 3456): True, (8192, 1152): True, (8192, 4608): True,            # PixArt-Sigma
+        (2048, 6720): True, (2048, 2240): False, (2048, 5600): True,           # SANA
+        (4096, 1280): True, (4096, 10240): True,                               # SDXL
+        (17776, 9216): True, (17776, 3072): True, (17776, 12288): True,        # CogVideoX
+        (256, 1152): False,
+    }
+    for (M, N), pair in faster_on_b200.items():
+        assert tasq.tasq_nvfp4_gemm_choice(M, N, 148) is pair, (M, N)
+    # a pair tile is 3x a one-CTA tile on half the slots: with the 1.1 time ratio the pair wins
+    # once the one-CTA kernel needs two waves more than 1.1x the pair's
+    for M, N in ((192, 256), (128, 128)):
+        assert tasq.tasq_nvfp4_gemm_choice(M, N, 148) is False
+    for bad in ((0, 8, 148), (8, 0, 148), (8, 8, 1)):
+        with pytest.raises(tasq.TasqError) as ei:
+            tasq.tasq_nvfp4_gemm_choice(*bad)
+        assert ei.value.status == tasq.TASQ_ERR_INVALID_ARG

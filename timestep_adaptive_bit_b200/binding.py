@@ -76,6 +76,7 @@ def _load():
         "tasq_debug_stuck_wait": [P, P],
         "tasq_debug_set_gemm_mode": [P, i32],
         "tasq_gemm_choice": [i64, i32, i32, ctypes.POINTER(i32)],
+        "tasq_nvfp4_gemm_choice": [i64, i32, i32, ctypes.POINTER(i32)],
         "tasq_nvfp4_scale_bytes": [i64, i32, ctypes.POINTER(i64)],
         "tasq_debug_quantize_nvfp4": [P, P, i64, i64, i32, P, P, P, P],
         "tasq_debug_nvfp4_weights": [P, i32, P, P, P],
@@ -281,6 +282,13 @@ def tasq_gemm_choice(M: int, N: int, num_sms: int) -> bool:
     """True when the automatic choice runs this GEMM on CTA pairs; host-only, needs no device."""
     pair = ctypes.c_int32(0)
     _check(lib.tasq_gemm_choice(int(M), int(N), int(num_sms), ctypes.byref(pair)))
+    return bool(pair.value)
+
+
+def tasq_nvfp4_gemm_choice(M: int, N: int, num_sms: int) -> bool:
+    """True when the automatic choice runs this NVFP4 GEMM on CTA pairs; host-only."""
+    pair = ctypes.c_int32(0)
+    _check(lib.tasq_nvfp4_gemm_choice(int(M), int(N), int(num_sms), ctypes.byref(pair)))
     return bool(pair.value)
 
 

@@ -1028,6 +1028,14 @@ tasq_status tasq_gemm_choice(int64_t M, int32_t N, int32_t num_sms, int32_t* pai
   return TASQ_OK;
 }
 
+tasq_status tasq_nvfp4_gemm_choice(int64_t M, int32_t N, int32_t num_sms, int32_t* pair) {
+  g_last_error.clear();
+  if (pair == nullptr) return fail(TASQ_ERR_INVALID_ARG, "pair is NULL");
+  if (M <= 0 || N <= 0 || num_sms <= 1) return fail(TASQ_ERR_INVALID_ARG, "M and N must be positive, num_sms > 1");
+  *pair = tasq::nvfp4_use_pair(M, N, num_sms) ? 1 : 0;
+  return TASQ_OK;
+}
+
 tasq_status tasq_debug_set_prologue_mode(tasq_ctx* c, int32_t mode) {
   g_last_error.clear();
   if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
