@@ -69,6 +69,8 @@ def parse_args(argv=None):
     p.add_argument("--nvfp4", action="store_true",
                    help="with --gemm-shape: time the block-scaled NVFP4 GEMM instead of the INT8 one; "
                         "with --sweep-bits: add an NVFP4 step (reported as width 0)")
+    p.add_argument("--dmpq-shape", default=None,
+                   help="M,D: time the on-device DMPQ predictor alone on one block input and output [M, D]")
     p.add_argument("--gemm-shape", default=None,
                    help="M,N,K: time the GEMM alone on given codes (one JSON line) and exit")
     p.add_argument("--graph", action="store_true",
@@ -499,6 +501,39 @@ def gemm_shape(args):
     return 0
 
 
+def dmpq_shape(args):
+    """CUDA-event time of tasq_dmpq_update alone on a synthetic block input and output [M, D]
+    (FP16, the output a small perturbation of the input), back to back."""
+    import torch
+    import timestep_adaptive_bit_b200 as T
+    M, D = (int(v) for v in args.dmpq_shape.split(","))
+    dev = torch.device("cuda:0")
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    x_in = torch.randn((M, D), device=dev, generator=g).to(torch.float16)
+    x_out = (x_in.float() + 0.05 * torch.randn((M, D), device=dev, generator=g)).to(torch.float16)
+    s = torch.cuda.current_stream()
+    w = torch.zeros((64, D), dtype=torch.int8, device=dev)
+    ctx = T.tasq_linear_create([(64, D, w, torch.ones(64, device=dev))], 1, 64, 16, T.TASQ_OUT_F16, s)
+    gamma = torch.zeros((1,), dtype=torch.float64, device=dev)
+    for _ in range(3):
+        T.tasq_dmpq_update(ctx, x_in, D, x_out, D, M, D, [0], 0, 0.05, 8, 4, gamma, s)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(args.reps):
+        T.tasq_dmpq_update(ctx, x_in, D, x_out, D, M, D, [0], 0, 0.05, 8, 4, gamma, s)
+    e1.record(s)
+    torch.cuda.synchronize()
+    us = 1e3 * e0.elapsed_time(e1) / args.reps
+    peaks, _ = load_peaks()
+    gbs = 4.0 * M * D / (us * 1e-6) / 1e9
+    print(json.dumps({"dmpq_shape": [M, D], "us": us, "gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                      "gamma": float(gamma.item()), "device_status": T.tasq_get_device_status(ctx)}), flush=True)
+    return 0
+
+
 def bitplanes(args):
     """The bit-plane formulation measured (TASQ's Temporal-Precision Engine streams only the kept
     weight bit planes, TASQ technical summary section 2). On B200 the only integer tensor-core
@@ -626,6 +661,8 @@ def main(argv=None):
         return sweep_bits(args)
     if args.gemm_shape:
         return gemm_shape(args)
+    if args.dmpq_shape:
+        return dmpq_shape(args)
     if args.bitplanes:
         return bitplanes(args)
 
