@@ -274,8 +274,9 @@ tasq_status tasq_debug_gemm_nvfp4(tasq_ctx* ctx, const void* codes, const void* 
  * CTA per 128 x 256 tile (tcgen05 cta_group::1), 2 forces CTA pairs on 256 x 256 tiles (tcgen05
  * cta_group::2). Both compute identical results. Any other mode is TASQ_ERR_INVALID_ARG.
  * The mode also selects the NVFP4 GEMM (forwards of NVFP4 steps and tasq_debug_gemm_nvfp4): 0
- * chooses by wave count, 1 forces one CTA per 128 x 128 tile, 2 forces CTA pairs on tiles of 256
- * channels x 128 tokens. Both NVFP4 kernels read the same code and scale layouts; their FP32
+ * chooses by wave count (tasq_nvfp4_gemm_choice), 1 forces one CTA per 128 x 128 tile, 2 forces
+ * CTA pairs on tiles of 256 channels x 192 tokens. Both NVFP4 kernels read the same code and
+ * scale layouts; their FP32
  * accumulators may differ in rounding order, each within the bound documented for
  * tasq_debug_gemm_nvfp4's raw accumulators.
  */
