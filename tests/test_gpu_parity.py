@@ -516,3 +516,60 @@ def test_trace_counts_launches(T):
     assert tr["gemm_launches"] == 4 and tr["prologue_launches"] == 4
     assert tr["gemm_ms"] > 0 and tr["prologue_ms"] > 0
     assert tr["gemm_ops"] == 4 * 2.0 * M * N * K
+
+
+def test_two_host_threads_two_contexts(T):
+    """Two host threads, each with its own context and stream, run INT8 and NVFP4 forwards at the
+    same time (run alone, both threads also reach the launchers' one-time per-device set-up of
+    shared-memory limits and resident CTA pairs together). Every output equals the oracle's: the
+    set-up is guarded, and contexts share no device state."""
+    import threading
+    n, M = 64, 700
+    shapes = [(1152, 4608), (4608, 1152)]        # the CTA-pair and the one-CTA INT8 GEMM
+    rng = np.random.default_rng(404)
+    jobs = []
+    for K, N in shapes:
+        w = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+        s_w = rng.uniform(0.001, 0.01, size=N).astype(np.float32)
+        jobs.append((K, N, w, s_w, _acts(rng, M, K)))
+    bits = [8, 5, 0, 3]                             # INT8 widths and an NVFP4 step
+    outs = [None, None]
+    errors = []
+
+    def run(i):
+        try:
+            K, N, w, s_w, x = jobs[i]
+            stream = torch.cuda.Stream()
+            ctx = T.tasq_linear_create([(N, K, w, s_w)], len(bits), n, M, 0, stream)
+            T.tasq_debug_set_gemm_mode(ctx, 2 if i == 0 else 1)
+            T.tasq_set_schedule(ctx, np.array([bits], np.uint8), stream)
+            xd = torch.from_numpy(x).cuda()
+            ys = []
+            for step in range(len(bits)):
+                y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+                T.tasq_linear_forward(ctx, xd, M, K, 0, step, y, N, stream)
+                ys.append(y)
+            stream.synchronize()
+            outs[i] = ([y.float().cpu().numpy().astype(np.float64) for y in ys], T.tasq_get_device_status(ctx))
+            T.tasq_linear_destroy(ctx)
+        except Exception as e:   # reported on the main thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=run, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=300)
+    assert not errors, errors
+    for i, (K, N, w, s_w, x) in enumerate(jobs):
+        ys, status = outs[i]
+        assert status == 0
+        for step, b in enumerate(bits):
+            if b == 0:
+                r4 = oracle.nvfp4_linear(x, w, s_w, n)
+                tol = (K * 2.0 ** -24 * oracle.nvfp4_abs_terms(r4["ca"], r4["sa"], r4["cw"], r4["sw"]) * 1.0001 *
+                       r4["s_x"][:, None] * s_w[None, :] + np.abs(r4["y"]) * (2.0 ** -11 + 2.0 ** -21) + ABS_TINY)
+                assert np.all(np.abs(ys[step] - r4["y"]) <= tol), f"thread {i} NVFP4 step"
+            else:
+                ref = oracle.masked_linear(x, w, s_w, b, n)["y"]
+                assert np.linalg.norm(ys[step] - ref) <= 1e-3 * np.linalg.norm(ref), f"thread {i} bits {b}"
