@@ -108,3 +108,60 @@ def test_fullsize_nvfp4_workload(T):
         assert T.tasq_get_device_status(ctx) == 0
         T.tasq_linear_destroy(ctx)
         del xd, y
+
+
+# (GEMM kernel, mask placement) pairs of the full-size INT32 check: kernel 1 = one CTA per
+# 128 x 256 tile, 2 = CTA pairs on 256 x 256 tiles; placement 1 = inside the GEMM, 2 = once ahead
+FULLSIZE_S32_MODES = [(1, 1), (1, 2), (2, 1), (2, 2)]
+
+
+@pytest.mark.parametrize("name", [w for w in workloads.WORKLOAD_ORDER if w != "single"])
+def test_fullsize_int32_accumulators_bit_exact(T, name):
+    """The raw INT32 accumulators of every distinct layer shape of a workload, at its full token
+    count and at every bit width its schedule uses, on both GEMM kernels and both mask placements,
+    equal the exact integer products of the GPU's own activation codes with the masked weights
+    (HQ-DM's integer core, section 2.1 "Eficiencia de Hardware"; TASQ's LSB mask, section 2).
+    These launches have many more tiles than CTAs, so every CTA walks several tiles through both
+    TMEM accumulators and both accumulator phases. Checked on the sampled rows (the whole last,
+    ragged token tile included) and every output channel."""
+    wl = workloads.WORKLOADS[name]
+    M, n = wl.tokens, wl.hadamard_n
+    sched = workloads.schedule(wl)
+    per = len(wl.block_layers)
+    picked, seen = [], set()
+    for j, (lname, K, N) in enumerate(wl.block_layers):
+        if (K, N) not in seen:
+            seen.add((K, N))
+            picked.append(j)
+    rows = workloads.sample_rows(M)
+    rows_d = torch.from_numpy(rows).cuda()
+    s = torch.cuda.current_stream()
+    for j in picked:
+        _, K, N = wl.layer_shape(j)
+        w, s_w = workloads.weights(wl, j)
+        x = workloads.activations(wl, j)
+        Kp = oracle.padded_k(K, n)
+        widths = sorted({int(v) for v in sched[j::per].ravel()} - {0}, reverse=True)
+        ctx = T.tasq_linear_create([(N, K, w, s_w)], 8, n, M, 0, s)
+        T.tasq_set_schedule(ctx, np.array([[8 - t for t in range(8)]], np.uint8), s)
+        xq = torch.empty((M, Kp), dtype=torch.int8, device="cuda")
+        sx = torch.empty((M,), dtype=torch.float32, device="cuda")
+        T.tasq_debug_quantize(ctx, torch.from_numpy(x).cuda(), M, K, 0, xq, sx, s)
+        torch.cuda.synchronize()
+        q_rows = xq[rows_d].cpu().numpy()
+        ld = N + (8 - N % 8) % 8
+        acc = torch.empty((M, ld), dtype=torch.int32, device="cuda")
+        for bits in widths:
+            ref = oracle.int_gemm(q_rows, oracle.lsb_mask(w, bits))
+            for gemm, mask in FULLSIZE_S32_MODES:
+                T.tasq_debug_set_gemm_mode(ctx, gemm)
+                T.tasq_debug_set_mask_mode(ctx, mask)
+                acc.fill_(0x7F7F7F7F)
+                T.tasq_debug_gemm_s32(ctx, xq, M, 0, 8 - bits, acc, ld, s)
+                torch.cuda.synchronize()
+                got = acc[rows_d, :N].cpu().numpy().astype(np.int64)
+                bad = np.argwhere(got != ref)
+                assert bad.size == 0, (name, K, N, bits, gemm, mask, bad[:4].tolist())
+        assert T.tasq_get_device_status(ctx) == 0
+        T.tasq_linear_destroy(ctx)
+        del xq, acc

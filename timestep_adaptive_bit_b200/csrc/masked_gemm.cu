@@ -17,8 +17,9 @@
 //                   stages of 128 bytes = four tcgen05.mma.kind::i8 of K = 32.
 //   warp 8          TMA producer: loads the 16 KB weight tile and the 32 KB code tile of each
 //                   stage into 128-byte-swizzled shared memory (4 stages in flight).
-//   warps 10-17     mask warps, two groups of four taking alternate K blocks (only when k > 0
-//                   and the weights were not masked ahead by the prologue launch): AND every
+//   warps 10-17     mask warps, two groups of four taking alternate K blocks (one group on the
+//                   3-stage ring of the INT32 test output; only when k > 0 and the weights were not
+//                   masked ahead by the prologue launch): AND every
 //                   weight byte of a landed stage with 0xFF << k in place (layout-agnostic,
 //                   8 x 16 B per thread), fence the generic-proxy writes to the async proxy and
 //                   release the stage to the MMA.
@@ -45,8 +46,17 @@ using namespace gemm;
 
 constexpr int kTileCh = kGemmTileCh;      // 128 output channels per tile
 constexpr int kABytes = kTileCh * kBlockK;
-constexpr int kMaskGroups = 2;            // groups of kMaskWarps mask warps, alternate K blocks
-constexpr int kThreads1 = kThreads + 32 * kMaskWarps * (kMaskGroups - 1);
+constexpr int kMaxMaskGroups = 2;         // groups of kMaskWarps mask warps, taking alternate K blocks
+constexpr int kThreads1 = kThreads + 32 * kMaskWarps * (kMaxMaskGroups - 1);
+
+// Mask groups of a ring of STAGES stages. A group waits for the `full` barrier of every G-th K block.
+// TMA loads may land out of order, so a group knows of no block's landing but its own: its parity
+// wait for block j is unambiguous only if block j - STAGES (the slot's previous phase) is one of its
+// own, i.e. STAGES is a multiple of G. The 4-stage ring takes two groups, the 3-stage one one.
+template <int STAGES>
+constexpr int mask_groups() {
+  return STAGES % kMaxMaskGroups == 0 ? kMaxMaskGroups : 1;
+}
 static_assert(kABytes % (16 * kMaskThreads) == 0, "mask pass must tile the weight stage");
 
 // Shared-memory plan of one instantiation: stages of (weights, codes), the epilogue's output
@@ -64,7 +74,8 @@ struct Plan {
   static constexpr int kSmemBytes = 1024 /* alignment slack */ + kBarOffset + kNumBars * 8 + 16;
   static_assert(kSmemBytes <= kMaxSmem, "shared memory");
   static_assert(kAccStages * kTok <= static_cast<int>(kTmemCols), "TMEM");
-  static_assert(kStages >= kMaskGroups, "one stage per mask group");
+  static constexpr int kMaskGroups = mask_groups<kStages>();
+  static_assert(kStages % kMaskGroups == 0, "a mask group's parity waits must stay unambiguous");
 };
 
 template <int STAGES>
@@ -227,7 +238,8 @@ __global__ void __launch_bounds__(kThreads1, 1)
   } else if (warp >= kMaskWarp0) {
     // -------------------------------------------------------------------- mask warps
     // Two groups of four warps take alternate K blocks of the CTA's sequence (group 0 the even
-    // ones), so that one group's load-mask-store latency overlaps the other's.
+    // ones), so that one group's load-mask-store latency overlaps the other's; with a 3-stage ring
+    // group 0 takes them all (see mask_groups).
     const int grp = (warp - kMaskWarp0) / kMaskWarps;
     const int t = threadIdx.x - (kMaskWarp0 + grp * kMaskWarps) * 32;
     // stage s of this group's next K block, and its phase
@@ -237,7 +249,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
     if (masking) {
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         for (int kb = 0; kb < g.num_kb; ++kb, ++seq) {
-          if (static_cast<int>(seq % kMaskGroups) != grp) continue;
+          if (static_cast<int>(seq % P::kMaskGroups) != grp) continue;
           if (!ptx::wait_bounded(bars.full(s), ph, limit, abort_flag)) {
             raise_failure(g.status, abort_flag, TASQ_DEVICE_TIMEOUT_MASK);
             ok = false;
@@ -247,7 +259,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
           ptx::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(bars.masked(s));
-          s += kMaskGroups;
+          s += P::kMaskGroups;
           if (s >= static_cast<uint32_t>(kStages)) {
             s -= kStages;
             ph ^= 1u;
