@@ -7,7 +7,10 @@ with the step's per-layer bit widths read from the device schedule table. Every 
 layer) has its own weights and its own activation buffer, so each step streams its whole
 input set from HBM (larger than L2).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload pixart] [--impl tasq|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload cogvideox] [--impl tasq|reference]
+
+The default workload is the largest one that fits a GPU, the CogVideoX-5B-shaped video DiT
+(17776 tokens, 42 blocks of {qkv 3072->9216, proj 3072->3072, fc1 3072->12288, fc2 12288->3072}).
 
 N > 1 runs under torchrun, one process per GPU, each an independent replica of the whole
 workload (the path shards along tokens with no exchange); the time is the max over ranks.
@@ -45,9 +48,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse_args(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=200)
-    p.add_argument("--warmup", type=int, default=10)
-    p.add_argument("--workload", default="pixart", choices=list(workloads.WORKLOADS))
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="cogvideox", choices=list(workloads.WORKLOADS))
+    p.add_argument("--no-int8-peak", action="store_true",
+                   help="skip the library INT8 GEMM peak measured beside the workload")
     p.add_argument("--impl", default="tasq", choices=["tasq", "reference"])
     p.add_argument("--out-dtype", default="f16", choices=["f16", "bf16"])
     p.add_argument("--no-e2e", action="store_true")
@@ -63,7 +68,8 @@ def parse_args(argv=None):
     p.add_argument("--gemm-mode", type=int, default=0, choices=[0, 1, 2],
                    help="GEMM kernel: 0 automatic, 1 one CTA per tile, 2 CTA pairs")
     p.add_argument("--mask-mode", type=int, default=0, choices=[0, 1, 2],
-                   help="LSB mask: 0 automatic, 1 inside the GEMM on every tile, 2 once ahead in the prologue launch")
+                   help="LSB mask: 0 in flight in the GEMM's weight feed (TMA at 8 bits), 1 in flight at every "
+                        "width, 2 once ahead in the prologue launch into a masked copy")
     p.add_argument("--bitplanes", default=None,
                    help="workload:layer -- time the bit-plane formulation against the masked dense GEMM")
     p.add_argument("--nvfp4", action="store_true",
@@ -135,6 +141,50 @@ def load_peaks():
         return d, "measured"
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def int8_library_peak(torch, device, sustain_s: float = 4.0, n: int = 8192):
+    """The tensor pipe's INT8 rate as a library reaches it on this GPU: torch._int_mm (cuBLASLt,
+    INT8 x INT8 -> INT32) at n^3, the best of 10 launches (burst) and the mean over about
+    sustain_s seconds of back-to-back launches (sustained, clocks sampled), the way the driver
+    measured its BF16 figures. 2 n^3 ops per launch."""
+    try:
+        g = torch.Generator(device=device)
+        g.manual_seed(0)
+        a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=device, generator=g)
+        b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=device, generator=g).t()
+        for _ in range(3):
+            torch._int_mm(a, b)
+        torch.cuda.synchronize()
+        best = None
+        for _ in range(10):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._int_mm(a, b)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        sampler = ClockSampler(device.index or 0)
+        sampler.start()
+        reps = max(1, int(sustain_s / (best / 1e3)))
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            torch._int_mm(a, b)
+        e1.record()
+        torch.cuda.synchronize()
+        clocks = sampler.stop()
+        sust_ms = e0.elapsed_time(e1) / reps
+        ops = 2.0 * n ** 3
+        return {"burst_tops": ops / (best / 1e3) / 1e12, "sustained_tops": ops / (sust_ms / 1e3) / 1e12,
+                "shape": [n, n, n], "library": "torch._int_mm (cuBLASLt INT8 -> INT32)",
+                "sustained_launches": reps, "sustained_clocks": clocks,
+                "datasheet_dense_tops": 4500.0}
+    except Exception as e:   # a library without an INT8 path here: report why, keep the bench line
+        return {"error": f"{type(e).__name__}: {str(e)[:200]}"}
 
 
 class ClockSampler:
@@ -814,7 +864,16 @@ def main(argv=None):
     value = total_ops / (ms_max / 1e3) / 1e12
     ms_per_step = ms_max / args.steps
     gemm_tops = trace["gemm_ops"] / (trace["gemm_ms"] / 1e3) / 1e12 if trace["gemm_ms"] > 0 else None
+    # the prologue's algorithmic bytes: activations only, M (2 K + Kp + 4) per launch; a weight pass
+    # (mask mode 2, or the NVFP4 steps' weight conversion) is reported apart
     pro_gbs = trace["prologue_bytes"] / (trace["prologue_ms"] / 1e3) / 1e9 if trace["prologue_ms"] > 0 else None
+    int8_lib = None
+    if not args.no_int8_peak:
+        int8_lib = int8_library_peak(torch, device)
+    # the kernel that runs most of the step's GEMM work with the automatic choice
+    big = max(wl.block_layers, key=lambda l: l[1] * l[2])
+    dominant = ("masked_gemm_pair_kernel" if T.tasq_gemm_choice(wl.tokens, big[2], torch.cuda.get_device_properties(
+        device).multi_processor_count) else "masked_gemm_kernel")
 
     if dist is not None:
         T.tasq_linear_destroy(ctx)
@@ -853,11 +912,20 @@ def main(argv=None):
                      "frac": (gemm_tops / int8_burst) if gemm_tops else None,
                      "traffic": profiled_traffic(wl.name),
                      "traffic_source": f"profiles/launches_{wl.name}_step.md (null once the GEMM sources change)",
-                     "kernel": "masked_gemm_kernel", "peak_kind": f"INT8 = 2 x {peak_kind} BF16 burst",
-                     "frac_of_sustained": (gemm_tops / int8_sust) if gemm_tops else None},
+                     "kernel": dominant, "peak_kind": f"INT8 = 2 x {peak_kind} BF16 burst",
+                     "frac_of_sustained": (gemm_tops / int8_sust) if gemm_tops else None,
+                     "int8_library": int8_lib,
+                     "frac_of_int8_library_burst": (gemm_tops / int8_lib["burst_tops"])
+                     if (gemm_tops and int8_lib and "burst_tops" in int8_lib) else None,
+                     "frac_of_int8_library_sustained": (gemm_tops / int8_lib["sustained_tops"])
+                     if (gemm_tops and int8_lib and "sustained_tops" in int8_lib) else None,
+                     "frac_of_datasheet_dense_int8": (gemm_tops / 4500.0) if gemm_tops else None},
         "prologue_roofline": {"bound": "hbm", "achieved": pro_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                               "frac": (pro_gbs / peaks["hbm_gbs"]) if pro_gbs else None,
                               "frac_of_8000": (pro_gbs / 8000.0) if pro_gbs else None,
+                              "bytes_per_step": trace["prologue_bytes"] / trace_steps,
+                              "bytes": "activations only: M (2 K + Kp + 4) per prologue launch",
+                              "weight_pass_bytes_per_step": trace["weight_pass_bytes"] / trace_steps,
                               "same_traffic_copy_gbs": copy_gbs,
                               "frac_of_same_traffic_copy": (pro_gbs / copy_gbs) if (pro_gbs and copy_gbs) else None},
         "gemm_share_of_step": trace["gemm_ms"] / max(traced_ms, 1e-9) if trace["gemm_ms"] else None,

@@ -84,8 +84,9 @@ typedef struct tasq_ctx tasq_ctx;
 /*
  * Create a context owning one shared weight buffer for `num_layers` layers, a device schedule
  * table bits[num_layers][num_steps] (every entry initialised to 8 = full precision), an
- * activation workspace for up to `max_tokens` tokens, and a transient buffer for masked
- * weights: min(num_layers, TASQ_GROUP_MAX) slots of the largest N x Kp of the layers.
+ * activation workspace for up to `max_tokens` tokens, and a transient weight buffer of
+ * min(num_layers, TASQ_GROUP_MAX) slots of the largest layer: an NVFP4 step's converted weights
+ * live there, and so do the masked copies that mask mode 2 (tasq_debug_set_mask_mode) makes.
  *   out         : receives the context; *out is set to NULL on failure.
  *   layers      : host array [num_layers] of layer descriptors.
  *   hadamard_n  : block size of the Hadamard transform along K, 64 or 128.
@@ -119,13 +120,12 @@ tasq_status tasq_set_schedule(tasq_ctx* ctx, const uint8_t* bits_host, void* str
  * Two kernels run on `stream`: the prologue (block Hadamard of size n along K with zero
  * padding to Kp, per-token absmax, s_x = absmax / (127 sqrt(n)), codes RNE(z * 127 / absmax)
  * in [-127, 127]) into the context workspace, then the GEMM, which accumulates exactly in INT32
- * and writes y = acc * s_x[m] * s_w[n]. The weights' low bit planes are cleared according to
- * bits[layer][step] read from the device table: when the last table given to
- * tasq_set_schedule drops bits for this (layer, step), the prologue launch writes the masked
- * layer into the context's masked-weight buffer once and the GEMM reads that; otherwise the
- * GEMM reads the stored weights and masks each tile in shared memory if the device table asks
- * for it. Uses the context workspace and masked-weight buffer: forwards of one context must not
- * overlap in time on different streams.
+ * and writes y = acc * s_x[m] * s_w[n]. The weights' low bit planes are cleared in flight,
+ * according to bits[layer][step] read from the device table: the GEMM loads every weight tile of
+ * the one stored buffer into shared memory and, when the step drops bits, its mask warps AND the
+ * tile with 0xFF << (8 - bits) there, before the tensor cores read it, so no masked copy of the
+ * weights is ever written. Uses the context workspace: forwards of one context must not overlap in
+ * time on different streams.
  */
 tasq_status tasq_linear_forward(tasq_ctx* ctx, const void* x, int64_t M, int64_t ldx, int32_t layer,
                                 int32_t step, void* y, int64_t ldy, void* stream);
@@ -139,9 +139,10 @@ tasq_status tasq_linear_forward(tasq_ctx* ctx, const void* x, int64_t M, int64_t
  *            min(num_layers, TASQ_GROUP_MAX).
  *   ys     : host array [count] of device output pointers; ldys : host array [count] of their
  *            row strides (elements, >= N of the layer, % 8 == 0).
- * The prologue launch masks the weights of every member whose step drops bits into its own slot
- * of the context's masked-weight buffer, which holds min(num_layers, TASQ_GROUP_MAX) slots. The
- * same overlap rule as tasq_linear_forward applies.
+ * Each GEMM masks its layer's weights in flight as tasq_linear_forward does (with mask mode 2 the
+ * prologue launch masks them ahead instead, each member into its own slot of the context's
+ * masked-weight buffer, which holds min(num_layers, TASQ_GROUP_MAX) slots). The same overlap rule
+ * as tasq_linear_forward applies.
  */
 tasq_status tasq_linear_forward_group(tasq_ctx* ctx, const void* x, int64_t M, int64_t ldx,
                                       const int32_t* layers, int32_t count, int32_t step, void* const* ys,
@@ -304,12 +305,15 @@ tasq_status tasq_nvfp4_gemm_choice(int64_t M, int32_t N, int32_t num_sms, int32_
 
 /*
  * Test hook: where later forwards (and tasq_debug_gemm / tasq_debug_gemm_s32) apply the step's
- * LSB mask to the weights (TASQ, "LSB masking" of the stored INT8 weights). 0 (default): ahead of
- * the GEMM, in the prologue launch, into a context-owned copy of the layer's weights whenever the
- * last schedule given to tasq_set_schedule has bits < 8 for the (layer, step), else inside the
- * GEMM; 1: always inside the GEMM, on every weight tile it loads; 2: always ahead. Every mode reads
- * the bit width from the device schedule table, so all give identical results for every table.
- * Any other mode is TASQ_ERR_INVALID_ARG.
+ * LSB mask to the weights (TASQ, "LSB masking" of the stored INT8 weights).
+ *   0 (default) and 1: in flight, inside the GEMM: its mask warps AND every weight tile of the
+ *     stored buffer with the step's byte mask in shared memory as it lands (no pass when the device
+ *     table keeps all 8 bits).
+ *   2: ahead of the GEMM, in the prologue launch, into a context-owned masked copy of the layer's
+ *     weights (2 N Kp bytes of extra traffic per forward) that the GEMM loads as it is; kept to
+ *     measure the in-flight mask against.
+ * Every mode reads the bit width from the device schedule table, so all give identical results
+ * for every table. Any other mode is TASQ_ERR_INVALID_ARG.
  */
 tasq_status tasq_debug_set_mask_mode(tasq_ctx* ctx, int32_t mode);
 
@@ -336,11 +340,20 @@ tasq_status tasq_debug_stuck_wait(tasq_ctx* ctx, void* stream);
  * records CUDA events around its prologue and GEMM kernels on the forward's stream, for up to
  * `capacity` forwards (later forwards are not recorded). tasq_trace_read synchronises the
  * recorded events and returns, per kernel kind, the number of launches and the summed
- * duration in milliseconds, then clears the trace. capacity 0 disables tracing.
+ * duration in milliseconds, then clears the trace. capacity 0 disables tracing. Any output
+ * pointer may be NULL.
+ *   gemm_ops          : 2 M N K integer ops of the recorded GEMMs (K unpadded).
+ *   prologue_bytes    : the prologue launches' activation bytes, M (2 K + Kp + 4) per launch
+ *                       (FP16 read, INT8 codes and FP32 scale written); NVFP4 steps count their
+ *                       codes and block scales instead.
+ *   weight_pass_bytes : bytes the same launches moved for weights: 2 N Kp per masked copy made
+ *                       ahead of the GEMM (tasq_debug_set_mask_mode 2 only), and the NVFP4 steps'
+ *                       weight conversion.
  */
 tasq_status tasq_trace_enable(tasq_ctx* ctx, int32_t capacity);
 tasq_status tasq_trace_read(tasq_ctx* ctx, int32_t* prologue_launches, double* prologue_ms,
-                            int32_t* gemm_launches, double* gemm_ms, double* gemm_ops, double* prologue_bytes);
+                            int32_t* gemm_launches, double* gemm_ms, double* gemm_ops, double* prologue_bytes,
+                            double* weight_pass_bytes);
 
 /*
  * Allocation-free variant of tasq_linear_forward, for callers that cannot call cudaMalloc:
@@ -359,19 +372,32 @@ tasq_status tasq_trace_read(tasq_ctx* ctx, int32_t* prologue_launches, double* p
  *   bits       : bit width for this call, 1..8 (8 = all bit planes kept).
  *   y          : device [M, N] in out_dtype, row stride ldy (>= N, % 8 == 0), 16-byte aligned.
  *   device_status : optional device uint32 that receives TASQ_DEVICE_* bits (OR-ed in; the
- *                caller clears it); NULL sends them to a word inside the fixed array.
- * Limits: (M * 4 rounded up to 1 KiB) + 256 + M * Kp must not exceed TASQ_NOALLOC_SCRATCH_BYTES;
- * larger sizes return TASQ_ERR_WORKSPACE before anything is enqueued.
+ *                caller clears it). With NULL the bits go to a status word inside the fixed array
+ *                instead, which the call clears first and tasq_noalloc_device_status reads.
+ * Limits: round_up(256 + 4 * M, 1024) + M * Kp bytes must not exceed TASQ_NOALLOC_SCRATCH_BYTES
+ * (a 256-byte control block and the M FP32 scales, rounded up to 1 KiB, then the M x Kp INT8
+ * codes); larger sizes return TASQ_ERR_WORKSPACE before anything is enqueued.
  * The first call on each device, made with that device current, looks the array's device
- * address up (cudaGetSymbolAddress) and caches it; make that first call before any stream
- * capture. Every call uses the same array and leaves its contents behind for the next one, so
- * calls that overlap on the GPU (on different streams, or from different threads without
- * ordering) race on it and must be serialised by the caller.
+ * address up (cudaGetSymbolAddress) and caches it with the CUDA context that was current; a
+ * later call under another context of the device (a non-primary driver context, or the primary
+ * context created again after cudaDeviceReset) looks it up again. Make the first call under each
+ * context before any stream capture. Every call uses the same array and leaves its contents
+ * behind for the next one, so calls that overlap on the GPU (on different streams, or from
+ * different threads without ordering) race on it and must be serialised by the caller.
  */
 #define TASQ_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 tasq_status tasq_linear_forward_noalloc(const void* x, int64_t M, int64_t ldx, int32_t K, const int8_t* w,
                                         const float* s_w, int32_t N, int32_t bits, int32_t hadamard_n, void* y,
                                         int64_t ldy, int32_t out_dtype, uint32_t* device_status, void* stream);
+
+/*
+ * The status word that tasq_linear_forward_noalloc calls made with device_status == NULL write
+ * on the current device: TASQ_DEVICE_* bits of the last such call (each one clears the word
+ * first), so that a caller without a device word of its own can still learn that a bounded wait
+ * ran out. Stream-ordered after the work enqueued on `stream`, which it synchronises; with clear
+ * non-zero the word is reset to 0 afterwards. Allocates nothing. The pages have no counterpart.
+ */
+tasq_status tasq_noalloc_device_status(uint32_t* status_out, int32_t clear, void* stream);
 
 #ifdef __cplusplus
 }

@@ -88,9 +88,10 @@ def _load():
         "tasq_debug_set_prologue_mode": [P, i32],
         "tasq_trace_enable": [P, i32],
         "tasq_linear_forward_noalloc": [P, i64, i64, i32, P, P, i32, i32, i32, P, i64, i32, P, P],
+        "tasq_noalloc_device_status": [ctypes.POINTER(ctypes.c_uint32), i32, P],
         "tasq_trace_read": [P, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i32),
                             ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
-                            ctypes.POINTER(ctypes.c_double)],
+                            ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)],
     }
     for name, args in sigs.items():
         f = getattr(lib, name)
@@ -310,11 +311,11 @@ def tasq_trace_enable(ctx: Context, capacity: int) -> None:
 
 def tasq_trace_read(ctx: Context) -> dict:
     pl, gl = ctypes.c_int32(), ctypes.c_int32()
-    pm, gm, ops, pb = ctypes.c_double(), ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+    pm, gm, ops, pb, wb = (ctypes.c_double() for _ in range(5))
     _check(lib.tasq_trace_read(ctx, ctypes.byref(pl), ctypes.byref(pm), ctypes.byref(gl), ctypes.byref(gm),
-                               ctypes.byref(ops), ctypes.byref(pb)))
+                               ctypes.byref(ops), ctypes.byref(pb), ctypes.byref(wb)))
     return {"prologue_launches": pl.value, "prologue_ms": pm.value, "gemm_launches": gl.value,
-            "gemm_ms": gm.value, "gemm_ops": ops.value, "prologue_bytes": pb.value}
+            "gemm_ms": gm.value, "gemm_ops": ops.value, "prologue_bytes": pb.value, "weight_pass_bytes": wb.value}
 
 
 def tasq_linear_forward_noalloc(x, M: int, ldx: int, K: int, w, s_w, N: int, bits: int, hadamard_n: int, y,
@@ -324,3 +325,10 @@ def tasq_linear_forward_noalloc(x, M: int, ldx: int, K: int, w, s_w, N: int, bit
     _check(lib.tasq_linear_forward_noalloc(_ptr(x), int(M), int(ldx), int(K), _ptr(w), _ptr(s_w), int(N), int(bits),
                                            int(hadamard_n), _ptr(y), int(ldy), int(out_dtype), _ptr(device_status),
                                            _stream(stream)))
+
+
+def tasq_noalloc_device_status(clear: bool = False, stream=None) -> int:
+    """Status word of the allocation-free calls made without a device status pointer."""
+    v = ctypes.c_uint32()
+    _check(lib.tasq_noalloc_device_status(ctypes.byref(v), 1 if clear else 0, _stream(stream)))
+    return int(v.value)

@@ -9,8 +9,12 @@
 // entry point itself calls no cudaMalloc, cudaFree or allocating library routine.
 //
 // Host code must not use the array's name as a device address (in host code it is a host-side
-// stand-in): the device address is fetched once per device with cudaGetSymbolAddress, on the
-// first call made with that device current, and cached.
+// stand-in): the device address is fetched with cudaGetSymbolAddress on the first call made with
+// a device current, and cached together with the CUDA context it belongs to. A call made under
+// another context of that device (a non-primary driver context, or the primary one created anew
+// after cudaDeviceReset, where the module and its array are loaded again) looks the address up
+// again instead of using a stale one.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -22,19 +26,53 @@
 
 namespace {
 
-// [0, 256): control block (byte 0: the bit width the GEMM reads; bytes 4..7: fallback status
-// word); [256, ...): per-token scales, then the INT8 codes at a 1024-byte aligned offset.
+// [0, 256): control block (byte 0: the bit width the GEMM reads; bytes 4..7: the status word of
+// calls made with device_status == NULL); [256, ...): per-token scales, then the INT8 codes at a
+// 1024-byte aligned offset.
 static __device__ __align__(256) unsigned char g_tasq_noalloc_scratch[TASQ_NOALLOC_SCRATCH_BYTES];
+
+constexpr size_t kSxOffset = 256;
+constexpr size_t kStatusOffset = 4;
+
+// Bytes of the array one call needs: the control block and M scales, rounded up to 1 KiB, then
+// M * Kp codes.
+size_t scratch_bytes(int64_t M, int32_t Kp) {
+  return tasq::round_up(kSxOffset + static_cast<size_t>(M) * sizeof(float), 1024) +
+         static_cast<size_t>(M) * static_cast<size_t>(Kp);
+}
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 unsigned char* g_scratch_ptr[kMaxDevices] = {nullptr};
+CUcontext g_scratch_ctx[kMaxDevices] = {nullptr};
 int g_num_sms[kMaxDevices] = {0};
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// The array's device address under the current context of device `dev` (and the device's SM
+// count), looked up on the first call under that context. A call with no context current yet gets
+// the runtime's primary context from the lookup itself.
 tasq_status device_setup(int dev, unsigned char** scratch, int* num_sms) {
   if (dev < 0 || dev >= kMaxDevices) return tasq::fail(TASQ_ERR_INVALID_ARG, "device index out of range");
+  CtxGetCurrentFn get = ctx_get_current();
+  if (get == nullptr) return tasq::fail(TASQ_ERR_CUDA, "cuCtxGetCurrent is not available from the driver");
+  CUcontext cur = nullptr;
+  if (get(&cur) != CUDA_SUCCESS) return tasq::fail(TASQ_ERR_CUDA, "cuCtxGetCurrent failed");
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (cur == nullptr || g_scratch_ptr[dev] == nullptr || g_scratch_ctx[dev] != cur) {
     cudaDeviceProp prop;
     cudaError_t e = cudaGetDeviceProperties(&prop, dev);
     if (e != cudaSuccess) return tasq::fail_cuda(e, "cudaGetDeviceProperties");
@@ -43,8 +81,10 @@ tasq_status device_setup(int dev, unsigned char** scratch, int* num_sms) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_tasq_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr) return tasq::fail_cuda(e, "cudaGetSymbolAddress(scratch)");
+    if (get(&cur) != CUDA_SUCCESS || cur == nullptr) return tasq::fail(TASQ_ERR_CUDA, "no current CUDA context");
     g_num_sms[dev] = prop.multiProcessorCount;
     g_scratch_ptr[dev] = static_cast<unsigned char*>(p);
+    g_scratch_ctx[dev] = cur;
   }
   *scratch = g_scratch_ptr[dev];
   *num_sms = g_num_sms[dev];
@@ -66,12 +106,12 @@ extern "C" tasq_status tasq_linear_forward_noalloc(const void* x, int64_t M, int
   if (M < 0 || M > 0x7fffffffLL) return fail(TASQ_ERR_INVALID_ARG, "M out of range");
   const int32_t Kp = (K + hadamard_n - 1) / hadamard_n * hadamard_n;
   if (Kp > TASQ_MAX_KP) return fail(TASQ_ERR_INVALID_ARG, "padded K exceeds TASQ_MAX_KP");
-  const size_t sx_off = 256;
-  const size_t xq_off = tasq::round_up(sx_off + static_cast<size_t>(M) * sizeof(float), 1024);
-  const size_t need = xq_off + static_cast<size_t>(M) * static_cast<size_t>(Kp);
+  const size_t xq_off = tasq::round_up(kSxOffset + static_cast<size_t>(M) * sizeof(float), 1024);
+  const size_t need = scratch_bytes(M, Kp);
   if (need > TASQ_NOALLOC_SCRATCH_BYTES)
-    return fail(TASQ_ERR_WORKSPACE, "M * Kp = " + std::to_string(static_cast<long long>(M) * Kp) +
-                                        " bytes of codes do not fit the fixed scratch of " +
+    return fail(TASQ_ERR_WORKSPACE, "M = " + std::to_string(static_cast<long long>(M)) + " tokens at Kp = " +
+                                        std::to_string(Kp) + " need " + std::to_string(need) +
+                                        " bytes of the fixed scratch of " +
                                         std::to_string(static_cast<unsigned long long>(TASQ_NOALLOC_SCRATCH_BYTES)) +
                                         " bytes");
   if (x == nullptr || !tasq::aligned16(x) || ldx < K || ldx % 8 != 0)
@@ -92,8 +132,9 @@ extern "C" tasq_status tasq_linear_forward_noalloc(const void* x, int64_t M, int
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   uint8_t* bits_byte = scratch;
-  uint32_t* status = device_status != nullptr ? device_status : reinterpret_cast<uint32_t*>(scratch + 4);
-  float* s_x = reinterpret_cast<float*>(scratch + sx_off);
+  uint32_t* status =
+      device_status != nullptr ? device_status : reinterpret_cast<uint32_t*>(scratch + kStatusOffset);
+  float* s_x = reinterpret_cast<float*>(scratch + kSxOffset);
   int8_t* xq = reinterpret_cast<int8_t*>(scratch + xq_off);
   // the array keeps the previous call's contents: set the bit width, clear the fallback status
   if ((e = cudaMemsetAsync(bits_byte, bits, 1, s)) != cudaSuccess) return tasq::fail_cuda(e, "set bit width");
@@ -113,7 +154,12 @@ extern "C" tasq_status tasq_linear_forward_noalloc(const void* x, int64_t M, int
   a.status = status;
   a.wait_limit_ns = 1000000000ull;
   a.num_sms = num_sms;
-  if ((e = tasq::launch_prologue(a, s)) != cudaSuccess) return tasq::fail_cuda(e, "prologue launch");
+  tasq::g_last_error.clear();
+  if ((e = tasq::launch_prologue(a, s)) != cudaSuccess) {
+    // the launcher may have left a more precise message (a failed per-device kernel set-up)
+    if (!tasq::g_last_error.empty()) return fail(TASQ_ERR_CUDA, "prologue launch: " + tasq::g_last_error);
+    return tasq::fail_cuda(e, "prologue launch");
+  }
 
   CUtensorMap tw, tx, ty;
   if ((st = tasq::make_tmap_u8(&tw, w, Kp, N, tasq::kGemmBlockK, tasq::kGemmTileCh)) != TASQ_OK) return st;
@@ -136,7 +182,33 @@ extern "C" tasq_status tasq_linear_forward_noalloc(const void* x, int64_t M, int
   g.ldy = ldy;
   g.status = status;
   g.wait_limit_ns = 1000000000ull;
+  // the caller's weights, masked in shared memory by the GEMM's mask warps as they land
   e = tasq::launch_masked_gemm(tw, tx, ty, g, bf16 ? tasq::OutKind::BF16 : tasq::OutKind::F16, num_sms, s);
   if (e != cudaSuccess) return tasq::fail_cuda(e, "masked GEMM launch");
+  return TASQ_OK;
+}
+
+extern "C" tasq_status tasq_noalloc_device_status(uint32_t* status_out, int32_t clear, void* stream) {
+  tasq::set_last_error("");
+  if (status_out == nullptr) return tasq::fail(TASQ_ERR_INVALID_ARG, "status_out is NULL");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return tasq::fail_cuda(e, "cudaGetDevice");
+  unsigned char* scratch = nullptr;
+  int num_sms = 0;
+  tasq_status st = device_setup(dev, &scratch, &num_sms);
+  if (st != TASQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* word = reinterpret_cast<uint32_t*>(scratch + kStatusOffset);
+  uint32_t v = 0;
+  e = cudaMemcpyAsync(&v, word, sizeof(v), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return tasq::fail_cuda(e, "read of the status word");
+  if (clear) {
+    e = cudaMemsetAsync(word, 0, sizeof(uint32_t), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return tasq::fail_cuda(e, "clear of the status word");
+  }
+  *status_out = v;
   return TASQ_OK;
 }

@@ -116,7 +116,7 @@ struct LayerInfo {
 
 struct TraceRec {
   cudaEvent_t e0, e1, e2;
-  double ops, bytes;
+  double ops, bytes, wbytes;   // GEMM ops, prologue activation bytes, weight-pass bytes
 };
 
 }  // namespace
@@ -142,7 +142,8 @@ struct tasq_ctx {
   float sx_factor = 0.0f;
   float sx_factor4 = 0.0f;              // NVFP4: fp32(1 / (2688 sqrt(n)))
   int32_t gemm_mode = 0;   // 0 automatic, 1 one CTA per tile, 2 CTA pairs
-  int32_t mask_mode = 0;   // 0 automatic, 1 mask inside the GEMM, 2 mask ahead in the prologue launch
+  int32_t mask_mode = 0;   // 0 and 1: in the GEMM, in shared memory; 2: ahead in the prologue launch,
+                           // into a masked copy
   int32_t prologue_mode = 0;   // 0 automatic, 1 direct-load prologue, 2 bulk-fed prologue where it fits
   // host copy of the last schedule given, used only to choose where the mask is applied: both
   // places read the device table and give the same result for every bit width, so a device table
@@ -225,13 +226,11 @@ tasq_status check_rows(const void* p, int64_t ld, int64_t width, const char* nam
   return TASQ_OK;
 }
 
-// Whether this forward masks the layer's weights once in the prologue launch (true) or lets the
-// GEMM mask every weight tile it loads (false). Masking ahead pays whenever the step drops bits;
-// at 8 bits the GEMM reads the stored weights directly.
-bool mask_ahead(const tasq_ctx* c, int32_t layer, int32_t step) {
-  if (c->mask_mode != 0) return c->mask_mode == 2;
-  return c->bits_host[static_cast<size_t>(layer) * c->num_steps + step] < 8;
-}
+// Whether this forward masks the layer's weights once in the prologue launch, into a masked copy
+// that the GEMM then loads (mask mode 2, kept to measure against). Otherwise the GEMM's mask warps
+// clear the step's low bit planes of every weight tile of the one stored buffer in shared memory, as
+// it lands, whenever the device table drops bits, and no copy of the weights exists.
+bool mask_ahead(const tasq_ctx* c, int32_t /*layer*/, int32_t /*step*/) { return c->mask_mode == 2; }
 
 int8_t* wk_slot(const tasq_ctx* c, int32_t slot) { return c->d_wk + static_cast<size_t>(slot) * c->wk_slot_bytes; }
 
@@ -669,7 +668,8 @@ tasq_status tasq_linear_forward(tasq_ctx* c, const void* x, int64_t M, int64_t l
     if (tr) {
       cudaEventRecord(tr->e2, s);
       tr->ops = 2.0 * static_cast<double>(M) * L.N * L.K;
-      tr->bytes = static_cast<double>(M) * (2.0 * L.K + L.Kp + 4.0) + (ahead ? 2.0 * L.N * L.Kp : 0.0);
+      tr->bytes = static_cast<double>(M) * (2.0 * L.K + L.Kp + 4.0);
+      tr->wbytes = ahead ? 2.0 * L.N * L.Kp : 0.0;
       ++c->trace_count;
     }
     return TASQ_OK;
@@ -686,8 +686,8 @@ tasq_status tasq_linear_forward(tasq_ctx* c, const void* x, int64_t M, int64_t l
     if (tr) {
       cudaEventRecord(tr->e2, s);
       tr->ops = 2.0 * static_cast<double>(M) * L.N * L.K;
-      tr->bytes = static_cast<double>(M) * (2.0 * L.K + L.Kp / 2.0 + L.Kp / 16.0 + 4.0) +
-                  static_cast<double>(L.N) * L.Kp * (1.0 + 0.5 + 1.0 / 16.0);
+      tr->bytes = static_cast<double>(M) * (2.0 * L.K + L.Kp / 2.0 + L.Kp / 16.0 + 4.0);
+      tr->wbytes = static_cast<double>(L.N) * L.Kp * (1.0 + 0.5 + 1.0 / 16.0);
       ++c->trace_count;
     }
     return TASQ_OK;
@@ -702,7 +702,8 @@ tasq_status tasq_linear_forward(tasq_ctx* c, const void* x, int64_t M, int64_t l
   if (tr) {
     cudaEventRecord(tr->e2, s);
     tr->ops = 2.0 * static_cast<double>(M) * L.N * L.K;
-    tr->bytes = static_cast<double>(M) * (2.0 * L.K + L.Kp + 4.0) + (ahead ? 2.0 * L.N * L.Kp : 0.0);
+    tr->bytes = static_cast<double>(M) * (2.0 * L.K + L.Kp + 4.0);
+    tr->wbytes = ahead ? 2.0 * L.N * L.Kp : 0.0;
     ++c->trace_count;
   }
   return TASQ_OK;
@@ -767,7 +768,8 @@ tasq_status tasq_linear_forward_group(tasq_ctx* c, const void* x, int64_t M, int
   if (tr) {
     cudaEventRecord(tr->e2, s);
     tr->ops = ops;
-    tr->bytes = static_cast<double>(M) * (2.0 * L0.K + L0.Kp + 4.0) + wbytes;
+    tr->bytes = static_cast<double>(M) * (2.0 * L0.K + L0.Kp + 4.0);
+    tr->wbytes = wbytes;
     ++c->trace_count;
   }
   return TASQ_OK;
@@ -1081,10 +1083,10 @@ tasq_status tasq_trace_enable(tasq_ctx* c, int32_t capacity) {
 }
 
 tasq_status tasq_trace_read(tasq_ctx* c, int32_t* prologue_launches, double* prologue_ms, int32_t* gemm_launches,
-                            double* gemm_ms, double* gemm_ops, double* prologue_bytes) {
+                            double* gemm_ms, double* gemm_ops, double* prologue_bytes, double* weight_pass_bytes) {
   g_last_error.clear();
   if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
-  double pm = 0, gm = 0, ops = 0, bytes = 0;
+  double pm = 0, gm = 0, ops = 0, bytes = 0, wbytes = 0;
   for (int32_t i = 0; i < c->trace_count; ++i) {
     TraceRec& r = c->trace[i];
     cudaError_t e = cudaEventSynchronize(r.e2);
@@ -1097,6 +1099,7 @@ tasq_status tasq_trace_read(tasq_ctx* c, int32_t* prologue_launches, double* pro
     gm += b;
     ops += r.ops;
     bytes += r.bytes;
+    wbytes += r.wbytes;
   }
   if (prologue_launches) *prologue_launches = c->trace_count;
   if (gemm_launches) *gemm_launches = c->trace_count;
@@ -1104,6 +1107,7 @@ tasq_status tasq_trace_read(tasq_ctx* c, int32_t* prologue_launches, double* pro
   if (gemm_ms) *gemm_ms = gm;
   if (gemm_ops) *gemm_ops = ops;
   if (prologue_bytes) *prologue_bytes = bytes;
+  if (weight_pass_bytes) *weight_pass_bytes = wbytes;
   c->trace_count = 0;
   return TASQ_OK;
 }
