@@ -35,6 +35,23 @@ struct OutTraits {
   static constexpr int kStageBytes = 32 * 32 * kBytes;   // one 32 x 32 output box per epilogue warp
 };
 
+// Order of a launch's tiles: bands of `band` token tiles (GemmArgs::band_tiles); inside a band the
+// token tile varies fastest, then the channel tile. The CTAs of one wave then work on a few token
+// tiles and a few channel tiles, and a band's codes stay in L2 while its channel tiles go by. With
+// the token tile varying fastest over all of M, every wave took all token tiles of one channel
+// tile, and once the codes outgrew L2 (CogVideoX fc2: 218 MB) they came from DRAM again for every
+// channel tile (2.5 GB read by one launch for 256 MB of operands). Every role of a kernel maps tile
+// indices the same way.
+__device__ __forceinline__ void tile_coords(int tile, int num_m_tiles, int num_n_tiles, int band, int& mt, int& nt) {
+  const int band_tiles = band * num_n_tiles;
+  const int b = tile / band_tiles;
+  const int within = tile - b * band_tiles;
+  const int m0 = b * band;
+  const int gm = num_m_tiles - m0 < band ? num_m_tiles - m0 : band;
+  mt = m0 + within % gm;
+  nt = within / gm;
+}
+
 __device__ __forceinline__ void raise_failure(uint32_t* status, volatile int* abort_flag, uint32_t bit) {
   atomicOr(status, bit);
   *abort_flag = 1;
@@ -101,8 +118,8 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
   // the token scales come from the prologue kernel just before this one
   ptx::grid_dep_wait();
   for (int tile = tile0; tile < num_tiles; tile += tile_step) {
-    const int mt = tile % g.num_m_tiles;
-    const int nt = tile / g.num_m_tiles;
+    int mt, nt;
+    tile_coords(tile, g.num_m_tiles, g.num_n_tiles, g.band_tiles, mt, nt);
     const int tok0 = mt * TOK + h * kEpiCols;
     const bool got = ptx::wait_bounded(acc_full + 8u * as, aph, limit, abort_flag);
     if (!__all_sync(0xffffffffu, got)) {

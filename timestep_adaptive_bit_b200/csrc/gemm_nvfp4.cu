@@ -127,8 +127,8 @@ __global__ void __launch_bounds__(kThreadsF4, 1)
       // the codes and scales come from the prologue kernel just before this one
       ptx::grid_dep_wait();
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int mt = tile % g.num_m_tiles;
-        const int nt = tile / g.num_m_tiles;
+        int mt, nt;
+        tile_coords(tile, g.num_m_tiles, g.num_n_tiles, g.band_tiles, mt, nt);
         const uint8_t* sfa_src = f.w_sf + (static_cast<int64_t>(nt) * f.sf_chunks) * kNvfp4ChunkBytes;
         const uint8_t* sfb_src = f.x_sf + (static_cast<int64_t>(mt) * f.sf_chunks) * kNvfp4ChunkBytes;
         for (int kb = 0; kb < g.num_kb; ++kb) {

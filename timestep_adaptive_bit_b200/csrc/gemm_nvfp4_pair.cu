@@ -210,8 +210,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsP4, 1)
       // the codes and scales come from the prologue kernel just before this one
       ptx::grid_dep_wait();
       for (int tile = pair_id; tile < num_tiles && ok; tile += num_pairs) {
-        const int mt = tile % g.num_m_tiles;
-        const int nt = tile / g.num_m_tiles;
+        int mt, nt;
+        tile_coords(tile, g.num_m_tiles, g.num_n_tiles, g.band_tiles, mt, nt);
         // this CTA's 128 weight rows; a group wholly past N has no scales to load (its rows are
         // zero-filled by the tensor map and its outputs are never stored), and likewise a token
         // group past the last token
@@ -315,7 +315,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsP4, 1)
     uint32_t s = 0, ph = 0;
     bool ok = true;
     for (int tile = pair_id; tile < num_tiles && ok; tile += num_pairs) {
-      const bool odd = (tile % g.num_m_tiles) & 1;
+      int mt, nt;
+      tile_coords(tile, g.num_m_tiles, g.num_n_tiles, g.band_tiles, mt, nt);
+      const bool odd = mt & 1;
       for (int kb = 0; kb < g.num_kb; ++kb) {
         const bool got = ptx::wait_bounded(bars.full(s), ph, limit, abort_flag);
         if (!__all_sync(0xffffffffu, got)) {

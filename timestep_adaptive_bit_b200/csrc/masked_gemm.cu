@@ -161,8 +161,8 @@ __global__ void __launch_bounds__(kThreads1, 1)
       // the activation codes come from the prologue kernel just before this one
       ptx::grid_dep_wait();
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int mt = tile % g.num_m_tiles;
-        const int nt = tile / g.num_m_tiles;
+        int mt, nt;
+        tile_coords(tile, g.num_m_tiles, g.num_n_tiles, g.band_tiles, mt, nt);
         for (int kb = 0; kb < g.num_kb; ++kb) {
           if (!ptx::wait_bounded(bars.empty(s), ph ^ 1u, limit, abort_flag)) {
             raise_failure(g.status, abort_flag, TASQ_DEVICE_TIMEOUT_PRODUCER);

@@ -144,8 +144,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // the activation codes come from the prologue kernel just before this one
       ptx::grid_dep_wait();
       for (int tile = pair_id; tile < num_tiles && ok; tile += num_pairs) {
-        const int mt = tile % g.num_m_tiles;
-        const int nt = tile / g.num_m_tiles;
+        int mt, nt;
+        tile_coords(tile, g.num_m_tiles, g.num_n_tiles, g.band_tiles, mt, nt);
         for (int kb = 0; kb < g.num_kb; ++kb) {
           // `empty` is arrived by the first CTA's tensor-core commit
           if (!ptx::wait_bounded(bars.empty(s), ph ^ 1u, limit, abort_flag)) {

@@ -174,6 +174,7 @@ extern "C" tasq_status tasq_linear_forward_noalloc(const void* x, int64_t M, int
   g.num_kb = (Kp + tasq::kGemmBlockK - 1) / tasq::kGemmBlockK;
   g.num_m_tiles = static_cast<int32_t>((M + tasq::kGemmTileTok - 1) / tasq::kGemmTileTok);
   g.num_n_tiles = (N + tasq::kGemmTileCh - 1) / tasq::kGemmTileCh;
+  g.band_tiles = tasq::gemm_band_tiles(g.num_m_tiles, tasq::kGemmTileTok, Kp);
   g.bits_table = bits_byte;
   g.bits_index = 0;
   g.s_x = s_x;

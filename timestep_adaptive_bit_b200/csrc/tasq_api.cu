@@ -374,6 +374,7 @@ tasq_status run_gemm_nvfp4(tasq_ctx* c, int32_t layer, int32_t step, const uint8
   g.status = c->d_status;
   g.wait_limit_ns = c->wait_limit_ns;
   g.gate = step < 0 ? tasq::kGateNone : gate;
+  g.band_tiles = tasq::gemm_band_tiles(g.num_m_tiles, tile_tok, L.Kp / 2);
   tasq::Nvfp4GemmArgs f{};
   f.w_sf = nvfp4_w_sf(c, layer, slot);
   f.x_sf = sf;
@@ -398,6 +399,16 @@ namespace tasq {
 // Narrower token tiles (64 .. 224 tokens, both kernels) were measured as well: a tile's time
 // shrinks much less than its width, so they lost everywhere but on a few wave-quantised shapes,
 // and won there by 3 % at most.
+// Bands of 8 token tiles. Measured on CogVideoX block 0 (DRAM bytes read per GEMM launch, ncu in
+// place): the token tile varying fastest over all of M read 228 / 84 / 299 / 2534 MB (qkv, proj,
+// fc1, fc2); bands of 8 read 170 / 63 / 351 / 654 MB; bands sized to keep 48 MB of codes in L2
+// (16 to 64 tiles) read 265 / 94 / 358 / 821 MB, the output stream evicting their codes.
+int32_t gemm_band_tiles(int64_t num_m_tiles, int64_t /*tile_tok*/, int64_t /*code_row_bytes*/) {
+  constexpr int64_t kBand = 8;
+  const int64_t band = num_m_tiles < kBand ? num_m_tiles : kBand;
+  return static_cast<int32_t>(band < 1 ? 1 : band);   // never 0: the kernels divide by it
+}
+
 bool gemm_use_pair(int64_t M, int64_t N, int num_sms) {
   const int64_t m_tiles = (M + kGemmTileTok - 1) / kGemmTileTok;
   const int64_t t1 = m_tiles * ((N + kGemmTileCh - 1) / kGemmTileCh);
@@ -459,6 +470,7 @@ tasq_status run_gemm(tasq_ctx* c, int32_t layer, int32_t step, const int8_t* xq,
   g.wait_limit_ns = c->wait_limit_ns;
   g.premasked = premasked ? 1 : 0;
   g.gate = gate;
+  g.band_tiles = tasq::gemm_band_tiles(g.num_m_tiles, tile_tok, L.Kp);
   CUtensorMap tw = premasked ? c->tmap_wk[layer] : c->tmap_w[layer];
   if (premasked && slot != 0) {
     st = make_tmap_u8(&tw, wk_slot(c, slot), static_cast<uint64_t>(L.Kp), static_cast<uint64_t>(L.N),

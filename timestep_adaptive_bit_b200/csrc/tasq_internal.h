@@ -151,7 +151,11 @@ struct GemmArgs {
   uint64_t wait_limit_ns;
   int32_t premasked;       // 1: the weight operand already holds mask(w) for this bit width
   int32_t gate;            // kGateNone, kGateInt8 or kGateNvfp4 (see gated_out), on bits_table[bits_index]
+  int32_t band_tiles;      // token tiles per band of the tile order (gemm_band_tiles), >= 1
 };
+// Token tiles per band of a GEMM's tile order (tile_coords): 8, or all token tiles when fewer, and
+// never 0.
+int32_t gemm_band_tiles(int64_t num_m_tiles, int64_t tile_tok, int64_t code_row_bytes);
 cudaError_t launch_masked_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const CUtensorMap& tmap_y,
                                const GemmArgs& g, OutKind out, int num_sms, cudaStream_t stream);
 
