@@ -81,8 +81,9 @@ def parse_args(argv=None):
                    help="M,N,K: time the GEMM alone on given codes (one JSON line) and exit")
     p.add_argument("--graph", action="store_true",
                    help="capture each schedule step's launches in a CUDA graph and time graph replays")
-    p.add_argument("--prologue-mode", type=int, default=0, choices=[0, 1, 2],
-                   help="prologue kernel: 0 automatic, 1 direct loads, 2 bulk-fed ring where it fits")
+    p.add_argument("--prologue-mode", type=int, default=0, choices=[0, 1, 2, 3],
+                   help="prologue kernel: 0 automatic, 1 direct loads (32 channels a thread), 2 bulk-fed ring "
+                        "where it fits, 3 direct loads with 64 channels a thread")
     return p.parse_args(argv)
 
 

@@ -321,9 +321,10 @@ tasq_status tasq_debug_set_mask_mode(tasq_ctx* ctx, int32_t mode);
  * Test hook: which prologue kernel later forwards and tasq_debug_quantize use. 1: the direct-load
  * kernel (each thread loads its 32 channels straight from global memory, one block of rows per
  * CTA); 2: the bulk-fed kernel (one persistent CTA per SM, rows streamed into a ring of
- * shared-memory stages by 1-D bulk copies) wherever its layout fits, else the direct one;
- * 0 (default): the bulk-fed kernel only when every SM gets many blocks of rows, else the direct
- * one. All produce bit-identical codes and scales. Any other mode is TASQ_ERR_INVALID_ARG.
+ * shared-memory stages by 1-D bulk copies) wherever its layout fits, else the direct one; 3: the
+ * direct-load kernel with 64 channels a thread; 0 (default): the 64-channel kernel for rows longer
+ * than 9216 channels (Kp), else the bulk-fed kernel when every SM gets many blocks of rows, else the
+ * direct one. All produce bit-identical codes and scales. Any other mode is TASQ_ERR_INVALID_ARG.
  */
 tasq_status tasq_debug_set_prologue_mode(tasq_ctx* ctx, int32_t mode);
 

@@ -63,8 +63,9 @@ def _ctx(T, layers, steps, n, max_tokens, out=0):
 
 
 # ----------------------------------------------------------------------------- prologue
-# prologue kernels: 1 = direct loads, 2 = bulk-fed ring wherever its layout fits
-@pytest.mark.parametrize("pmode", [1, 2])
+# prologue kernels: 1 = direct loads (32 channels a thread), 2 = bulk-fed ring wherever its layout
+# fits, 3 = direct loads with 64 channels a thread
+@pytest.mark.parametrize("pmode", [1, 2, 3])
 @pytest.mark.parametrize("n,K,M", [(64, 64, 1), (64, 96, 3), (64, 1152, 257), (128, 2240, 130), (128, 128, 5),
                                    (64, 12288, 33), (128, 16384, 2), (64, 4608, 300), (128, 5600, 64),
                                    (64, 1152, 4000), (64, 640, 9001), (128, 3072, 1500)])
@@ -102,7 +103,7 @@ def test_prologue_matches_oracle(T, n, K, M, pmode):
 # 254 once and small odd integers elsewhere, so a = 254, fp32(127 / a) = 0.5 and every other
 # z * 0.5 is a half-integer. x = z H_n / n is a multiple of 1/n below 2^11 / n, exact in FP16, and
 # every butterfly sum of it is exact in FP32, so both sides see the same exact ties.
-@pytest.mark.parametrize("pmode", [1, 2])
+@pytest.mark.parametrize("pmode", [1, 2, 3])
 @pytest.mark.parametrize("n,blocks,M", [(64, 3, 37), (128, 2, 20), (64, 18, 600)])
 def test_prologue_exact_ties_round_to_even(T, n, blocks, M, pmode):
     rng = np.random.default_rng(n * 1000 + blocks * 10 + M)
@@ -470,7 +471,7 @@ def test_argument_errors_on_device(T):
     assert err(T.tasq_debug_set_gemm_mode, ctx, 3) == T.TASQ_ERR_INVALID_ARG
     assert err(T.tasq_debug_set_mask_mode, ctx, 3) == T.TASQ_ERR_INVALID_ARG
     assert err(T.tasq_debug_set_mask_mode, ctx, -1) == T.TASQ_ERR_INVALID_ARG
-    assert err(T.tasq_debug_set_prologue_mode, ctx, 3) == T.TASQ_ERR_INVALID_ARG
+    assert err(T.tasq_debug_set_prologue_mode, ctx, 4) == T.TASQ_ERR_INVALID_ARG
     T.tasq_linear_forward(ctx, x, 0, K, 0, 0, y, N, s)        # M = 0: nothing to do
     assert T.tasq_get_device_status(ctx) == 0
     with pytest.raises(T.TasqError):

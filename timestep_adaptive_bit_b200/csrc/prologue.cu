@@ -18,13 +18,15 @@
 // produces. The per-row absmax is combined through a shared-memory atomicMax on the float bits
 // (all values are non-negative). No FMA contraction happens anywhere on the path.
 //
-// Two variants compute the same bits:
+// Three variants compute the same bits:
 //   bulk-fed  one persistent CTA per SM; a producer warp streams blocks of rows into a ring of
 //             shared-memory stages, one 1-D bulk copy per row, so that many bytes stay in flight
 //             while up to 31 compute warps work on the stages already landed (any K % 8 == 0).
 //   direct    a CTA owns R consecutive rows and R * Kp / 32 threads that load their 64 bytes
 //             straight from global memory (two full sectors) and store 32 (one sector); it
 //             serves the weight-only launch and arguments the bulk-fed layout does not fit.
+//   direct64  the same with 64 channels (128 bytes) a thread, R * Kp / 64 threads a CTA: for
+//             n = 64 a whole Hadamard block in one thread; taken for rows longer than 9216.
 //
 // The same launch can also truncate a layer's weights for the step (TASQ's LSB mask,
 // w AND (0xFF << k) with k = 8 - bits) into a masked copy that the GEMM then reads as its weight
@@ -307,6 +309,160 @@ __global__ void __launch_bounds__(MAXT, MINB)
   } else {
     st_16B(dst, w[0], w[1], w[2], w[3]);
     st_16B(dst + 16, w[4], w[5], w[6], w[7]);
+  }
+  if (seg == 0) a.s_x[row] = __fmul_rn(amax, a.sx_factor);
+}
+
+// ------------------------------------------------------------------------------ 64 channels a thread
+// The same arithmetic with 64 consecutive channels per thread: for n = 64 a thread holds a whole
+// Hadamard block, so every butterfly stage stays in registers (no shuffle), and the per-thread
+// costs (addressing, the row's absmax, the division) are spread over twice the elements. The 64
+// values sit in 32 register pairs, pair p = (z_p, z_(p+32)): strides 1 .. 16 are packed FP32x2
+// add / fma between pairs, stride 32 runs inside each pair; for n = 128 the stride-64 stage pairs
+// the two threads of a block through one xor shuffle. The stages run in increasing stride, each
+// butterfly rounded once in FP32, exactly as in the 32-channel kernel.
+
+// u[i] holds channels 2i, 2i + 1 (FP16) -> v[p] = (z_p, z_(p+32)) in FP32 (exact).
+__device__ __forceinline__ void to_pairs64(const uint32_t (&u)[32], float2 (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    __half2 hl, hh;
+    *reinterpret_cast<uint32_t*>(&hl) = u[i];        // channels 2i, 2i + 1
+    *reinterpret_cast<uint32_t*>(&hh) = u[i + 16];   // channels 32 + 2i, 33 + 2i
+    const float2 fl = __half22float2(hl);
+    const float2 fh = __half22float2(hh);
+    v[2 * i] = make_float2(fl.x, fh.x);
+    v[2 * i + 1] = make_float2(fl.y, fh.y);
+  }
+}
+
+template <bool N128>
+__device__ __forceinline__ void fwht_segment64(float2 (&v)[32], int seg) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int p = 0; p < 32; ++p) {
+      if ((p & h) == 0) butterfly2(v[p], v[p + h]);
+    }
+  }
+#pragma unroll
+  for (int p = 0; p < 32; ++p) {
+    const float lo = v[p].x, hi = v[p].y;
+    v[p].x = __fadd_rn(lo, hi);
+    v[p].y = __fsub_rn(lo, hi);
+  }
+  if constexpr (N128) {
+    // stride 64: the lower segment of the block keeps mine + other, the upper one other - mine
+    const float sgn = (seg & 1) != 0 ? -1.0f : 1.0f;
+#pragma unroll
+    for (int p = 0; p < 32; ++p) {
+      float2 o;
+      o.x = __shfl_xor_sync(0xffffffffu, v[p].x, 1);
+      o.y = __shfl_xor_sync(0xffffffffu, v[p].y, 1);
+      v[p] = fma2_sign(v[p], sgn, o);
+    }
+  }
+}
+
+__device__ __forceinline__ float absmax_segment64(const float2 (&v)[32]) {
+  float mx = 0.0f;
+#pragma unroll
+  for (int p = 0; p < 32; ++p) mx = fmaxf(mx, fmaxf(fabsf(v[p].x), fabsf(v[p].y)));
+  return mx;
+}
+
+// Codes of the 64 channels: w[j] = channels 4j .. 4j + 3 (j < 8 from the .x halves, j >= 8 the
+// .y halves), the lowest channel in the lowest byte.
+__device__ __forceinline__ void codes_segment64(float2 (&v)[32], float inv, uint32_t (&w)[16]) {
+#pragma unroll
+  for (int p = 0; p < 32; ++p) v[p] = mul2(v[p], inv);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    w[j] = pack4(code(v[4 * j].x), code(v[4 * j + 1].x), code(v[4 * j + 2].x), code(v[4 * j + 3].x));
+    w[8 + j] = pack4(code(v[4 * j].y), code(v[4 * j + 1].y), code(v[4 * j + 2].y), code(v[4 * j + 3].y));
+  }
+}
+
+// N128: n = 128 (two threads per Hadamard block); VEC32: rows of x and xq 32-byte aligned. A CTA
+// owns rows_per_cta rows of Kp / 64 threads each; CTAs [row_ctas, gridDim) run the weight pass.
+template <bool N128, bool VEC32, int MAXT, int MINB>
+__global__ void __launch_bounds__(MAXT, MINB)
+    prologue64_kernel(const PrologueArgs a, const int rows_per_cta, const int row_ctas) {
+  if (gated_out(a.gate, a.bits_table, a.gate_index)) return;
+  if (static_cast<int>(blockIdx.x) >= row_ctas) {
+    weight_pass(a, blockIdx.x - row_ctas, gridDim.x - row_ctas);
+    return;
+  }
+  const int L = a.Kp >> 6;                       // 64-channel segments per row
+  const int tid = threadIdx.x;
+  const int r_local = tid / L;
+  const int seg = tid - r_local * L;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + r_local;
+  const bool active = r_local < rows_per_cta && row < a.M;
+
+  // x may be the previous kernel's output: wait for it, then let the GEMM start its setup
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  __shared__ unsigned int row_max[kMaxRowsPerCta];
+  if (tid < rows_per_cta) row_max[tid] = 0u;
+  __syncthreads();
+
+  const int c0 = seg * 64;
+  float2 v[32];
+  {
+    uint32_t u[32];   // u[i] holds channels c0 + 2i, c0 + 2i + 1
+    const __half* src = static_cast<const __half*>(a.x) + row * a.ldx + c0;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      uint32_t* ug = u + 8 * g;
+      const int e0 = c0 + 16 * g;
+      if (active && e0 + 16 <= a.K) {
+        if constexpr (VEC32) {
+          uint32_t t[8];
+          ld_32B(src + 16 * g, t);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) ug[i] = t[i];
+        } else {
+          const uint4 p0 = ld_16B(src + 16 * g), p1 = ld_16B(src + 16 * g + 8);
+          ug[0] = p0.x; ug[1] = p0.y; ug[2] = p0.z; ug[3] = p0.w;
+          ug[4] = p1.x; ug[5] = p1.y; ug[6] = p1.z; ug[7] = p1.w;
+        }
+      } else if (active && e0 + 8 <= a.K) {
+        const uint4 p0 = ld_16B(src + 16 * g);
+        ug[0] = p0.x; ug[1] = p0.y; ug[2] = p0.z; ug[3] = p0.w;
+        ug[4] = 0u; ug[5] = 0u; ug[6] = 0u; ug[7] = 0u;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ug[i] = 0u;
+      }
+    }
+    to_pairs64(u, v);
+  }
+  fwht_segment64<N128>(v, seg);
+  const float mx = absmax_segment64(v);
+  if (active) atomicMax(&row_max[r_local], __float_as_uint(mx));
+  __syncthreads();
+  if (!active) return;
+  const float amax = __uint_as_float(row_max[r_local]);
+  const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+  uint32_t w[16];
+  codes_segment64(v, inv, w);
+  int8_t* dst = a.xq + row * a.Kp + c0;
+  if constexpr (VEC32) {
+    uint32_t w0[8], w1[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      w0[i] = w[i];
+      w1[i] = w[8 + i];
+    }
+    st_32B(dst, w0);
+    st_32B(dst + 32, w1);
+  } else {
+    st_16B(dst, w[0], w[1], w[2], w[3]);
+    st_16B(dst + 16, w[4], w[5], w[6], w[7]);
+    st_16B(dst + 32, w[8], w[9], w[10], w[11]);
+    st_16B(dst + 48, w[12], w[13], w[14], w[15]);
   }
   if (seg == 0) a.s_x[row] = __fmul_rn(amax, a.sx_factor);
 }
@@ -807,6 +963,53 @@ bool try_launch_fed(const PrologueArgs& a, cudaStream_t stream, cudaError_t* err
 
 }  // namespace
 
+namespace {
+
+// The 64-channel direct kernel: rows of Kp / 64 threads, CTAs of up to k64Threads threads.
+constexpr int k64Threads = 256;
+constexpr int k64MinBlocks = 3;
+
+cudaError_t launch_prologue64(const PrologueArgs& a, int64_t w_bytes, cudaStream_t stream) {
+  const bool weights = a.num_w > 0;
+  const int L = a.Kp / 64;
+  if (L > k64Threads) return cudaErrorInvalidValue;
+  int R = 1, threads = 128;
+  int64_t row_ctas = 0;
+  if (a.M > 0) {
+    R = pick_rows(L, k64Threads);
+    threads = ((R * L + 31) / 32) * 32;
+    row_ctas = (a.M + R - 1) / R;
+  }
+  int64_t weight_ctas = 0;
+  if (weights) {
+    const int64_t per_cta = static_cast<int64_t>(threads) * 32 * kWeightUnroll;
+    weight_ctas = (w_bytes + per_cta - 1) / per_cta;
+    if (weight_ctas > kMaxWeightCtas) weight_ctas = kMaxWeightCtas;
+  }
+  const int64_t grid = row_ctas + weight_ctas;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const bool vec32 = a.M > 0 && (reinterpret_cast<uintptr_t>(a.x) % 32 == 0) && (a.ldx % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(a.xq) % 32 == 0);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = use_pdl() ? 1 : 0;
+  const int rc = static_cast<int>(row_ctas);
+  if (a.n == 64) {
+    if (vec32) return cudaLaunchKernelEx(&cfg, prologue64_kernel<false, true, k64Threads, k64MinBlocks>, a, R, rc);
+    return cudaLaunchKernelEx(&cfg, prologue64_kernel<false, false, k64Threads, k64MinBlocks>, a, R, rc);
+  }
+  if (vec32) return cudaLaunchKernelEx(&cfg, prologue64_kernel<true, true, k64Threads, k64MinBlocks>, a, R, rc);
+  return cudaLaunchKernelEx(&cfg, prologue64_kernel<true, false, k64Threads, k64MinBlocks>, a, R, rc);
+}
+
+}  // namespace
+
 cudaError_t launch_prologue_nvfp4(const Nvfp4PrologueArgs& a, cudaStream_t stream) {
   const bool weights = a.w != nullptr;
   if (a.M <= 0 && !weights) return cudaSuccess;
@@ -876,7 +1079,14 @@ cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
     w_bytes += ws.bytes;
   }
   if (weights && (a.bits_table == nullptr || a.status == nullptr)) return cudaErrorInvalidValue;
-  if (a.variant != 1) {
+  // Rows longer than kSmallThreads 32-channel segments (Kp > 9216) take the 64-channel kernel:
+  // with 32 channels a thread a row needs the 512-thread instance at one CTA per SM, with 64 it is
+  // 192 threads for K = 12288 and four CTAs share an SM (CogVideoX fc2, 17776 x 12288: 123-132 us
+  // against 150-164 for the bulk-fed kernel and 159-173 for the 32-channel one). On shorter rows
+  // the 64-channel kernel ran level with the 32-channel one or behind it.
+  if (a.variant == 3 || (a.variant == 0 && a.M > 0 && a.Kp / 32 > kSmallThreads))
+    return launch_prologue64(a, w_bytes, stream);
+  if (a.variant == 0 || a.variant == 2) {
     cudaError_t e = cudaSuccess;
     if (try_launch_fed(a, stream, &e)) return e;
   }

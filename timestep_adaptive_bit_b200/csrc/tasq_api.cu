@@ -144,7 +144,8 @@ struct tasq_ctx {
   int32_t gemm_mode = 0;   // 0 automatic, 1 one CTA per tile, 2 CTA pairs
   int32_t mask_mode = 0;   // 0 and 1: in the GEMM, in shared memory; 2: ahead in the prologue launch,
                            // into a masked copy
-  int32_t prologue_mode = 0;   // 0 automatic, 1 direct-load prologue, 2 bulk-fed prologue where it fits
+  int32_t prologue_mode = 0;   // 0 automatic, 1 direct-load prologue, 2 bulk-fed prologue where it fits,
+                               // 3 direct-load prologue with 64 channels a thread
   // host copy of the last schedule given, used only to choose where the mask is applied: both
   // places read the device table and give the same result for every bit width, so a device table
   // that is newer or older than this copy changes no result
@@ -1053,7 +1054,7 @@ tasq_status tasq_nvfp4_gemm_choice(int64_t M, int32_t N, int32_t num_sms, int32_
 tasq_status tasq_debug_set_prologue_mode(tasq_ctx* c, int32_t mode) {
   g_last_error.clear();
   if (c == nullptr) return fail(TASQ_ERR_INVALID_ARG, "ctx is NULL");
-  if (mode < 0 || mode > 2) return fail(TASQ_ERR_INVALID_ARG, "mode must be 0, 1 or 2");
+  if (mode < 0 || mode > 3) return fail(TASQ_ERR_INVALID_ARG, "mode must be 0, 1, 2 or 3");
   c->prologue_mode = mode;
   return TASQ_OK;
 }
