@@ -274,18 +274,20 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
   if (lane == 0) ptx::bulk_wait0();
 }
 
-// In-place LSB mask of one landed weight stage: every byte AND (0xFF << k), 16 bytes at a time.
-template <int A_BYTES>
+// In-place LSB mask of one landed weight stage by THREADS threads (thread t of them): every byte
+// AND (0xFF << k), 16 bytes at a time.
+template <int A_BYTES, int THREADS = kMaskThreads>
 __device__ __forceinline__ void mask_stage(uint8_t* a_stage, int t, uint32_t mask32) {
+  static_assert(A_BYTES % (16 * THREADS) == 0, "mask pass must tile the weight stage");
   uint4* wt = reinterpret_cast<uint4*>(a_stage);
 #pragma unroll
-  for (int i = 0; i < A_BYTES / 16 / kMaskThreads; ++i) {
-    uint4 w = wt[i * kMaskThreads + t];
+  for (int i = 0; i < A_BYTES / 16 / THREADS; ++i) {
+    uint4 w = wt[i * THREADS + t];
     w.x &= mask32;
     w.y &= mask32;
     w.z &= mask32;
     w.w &= mask32;
-    wt[i * kMaskThreads + t] = w;
+    wt[i * THREADS + t] = w;
   }
 }
 

@@ -9,9 +9,9 @@
 // channels x 256 tokens. Per SM and per K stage this moves half the activation bytes of the
 // one-CTA tile through shared memory and L2 for the same number of MACs.
 //
-// Roles per CTA (448 threads), as in the one-CTA kernel but with one group of mask warps:
+// Roles per CTA (576 threads), as in the one-CTA kernel but with one group of eight mask warps:
 //   warp 8      TMA producer of this CTA's halves, completion on its own `full` barrier.
-//   warps 10-13 apply the step's LSB mask to this CTA's weight half in place (when k > 0 and the
+//   warps 10-17 apply the step's LSB mask to this CTA's weight half in place (when k > 0 and the
 //               weights were not masked ahead by the prologue launch) and then arrive on the
 //               first CTA's `ready` barrier (one arrival per warp).
 //   warp 9      TMEM allocation for the pair (both CTAs); in the first CTA also the MMA thread,
@@ -40,7 +40,11 @@ constexpr int kABytes = kHalf * kBlockK;  // 16 KB
 constexpr int kBBytes = kHalf * kBlockK;  // 16 KB
 constexpr int kStageBytes = kABytes + kBBytes;
 static_assert(kPairTok == kAccCols, "accumulator width");
-static_assert(kABytes % (16 * kMaskThreads) == 0, "mask pass must tile the weight stage");
+// Eight mask / relay warps (10-17): the in-place pass of a stage, on the path from its landing to
+// its MMA, takes half as long as with four (masked CogVideoX GEMMs 4-11 % faster; the one-CTA
+// kernel is better served by two alternating groups of four).
+constexpr int kPairMaskWarps = 8;
+constexpr int kPairThreads = 32 * (kMaskWarp0 + kPairMaskWarps);
 
 template <int OUT>
 struct PairPlan {
@@ -66,7 +70,7 @@ struct PairBars {
 };
 
 template <int OUT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     masked_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                             const __grid_constant__ CUtensorMap tmap_y, const GemmArgs g) {
   using P = PairPlan<OUT>;
@@ -101,7 +105,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(bars.full(s), 1);
-      ptx::mbar_init(bars.ready(s), 2 * kMaskWarps);
+      ptx::mbar_init(bars.ready(s), 2 * kPairMaskWarps);
       ptx::mbar_init(bars.empty(s), 1);
     }
     for (int i = 0; i < kAccStages; ++i) {
@@ -236,7 +240,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           break;
         }
         if (masking) {
-          mask_stage<kABytes>(smem + s * kABytes, t, mask32);
+          mask_stage<kABytes, 32 * kPairMaskWarps>(smem + s * kABytes, t, mask32);
           ptx::fence_proxy_async_smem();
         }
         // one arrival per warp on the first CTA's barrier (remote arrivals are not free)
@@ -293,7 +297,7 @@ cudaError_t launch_pair_out(const CUtensorMap& tw, const CUtensorMap& tx, const 
       // how many CTA pairs can be resident at once on this device
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
-      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.blockDim = dim3(kPairThreads, 1, 1);
       cfg.dynamicSmemBytes = PairPlan<OUT>::kSmemBytes;
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -320,7 +324,7 @@ cudaError_t launch_pair_out(const CUtensorMap& tw, const CUtensorMap& tx, const 
   const int pairs = tiles < resident_pairs ? tiles : resident_pairs;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(kPairThreads, 1, 1);
   cfg.dynamicSmemBytes = PairPlan<OUT>::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
