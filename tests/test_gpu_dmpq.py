@@ -105,6 +105,35 @@ def test_zero_input_and_extremes(T):
     assert table[0, 1] == 8 and table[1, 1] == 6 and table[2, 1] == 8
 
 
+def _all_finite_fp16(rng, max_exponent_field=30):
+    """Every finite FP16 bit pattern whose exponent field is at most max_exponent_field (both
+    signs, both zeros), in random order."""
+    h = np.arange(65536, dtype=np.uint32)
+    h = h[((h >> 10) & 31) <= max_exponent_field]
+    return rng.permutation(h).astype(np.uint16).view(np.float16)
+
+
+def test_every_finite_fp16_value_enters_the_sums_exactly(T):
+    """Input and output each hold every finite FP16 value once (63488 patterns as 248 x 256), in
+    two different orders; then only subnormals and the smallest normals (|x| < 2^-11, 8192
+    patterns), where both sums stay below 2^53 units: Gamma is then the quotient of two exact
+    doubles, and one unit more or less in either sum changes it."""
+    rng = np.random.default_rng(17)
+    ctx = _ctx(T, 2, 1)
+    g = torch.zeros((1,), dtype=torch.float64, device="cuda")
+    for idx, (max_e, M, D) in enumerate([(30, 248, 256), (3, 32, 256)]):
+        x_in = _all_finite_fp16(rng, max_e).reshape(M, D)
+        x_out = _all_finite_fp16(rng, max_e).reshape(M, D)
+        T.tasq_dmpq_update(ctx, torch.from_numpy(x_in).cuda(), D, torch.from_numpy(x_out).cuda(), D, M, D, [idx],
+                           0, 0.5, 8, 4, g, _s())
+        num, den = oracle.dmpq_l1_sums(x_in, x_out)
+        if max_e == 3:
+            assert num < 2 ** 53 and den < 2 ** 53
+            assert float(num + 1) / float(den) != float(num) / float(den)
+        assert float(g.item()) == oracle.dmpq_gamma(x_in, x_out), max_e
+    assert T.tasq_get_device_status(ctx) == 0
+
+
 def test_full_size_sums_stay_exact(T):
     """CogVideoX-sized block (17776 x 3072) at the largest magnitudes: the exact sums exceed 2^64
     units, which the 128-bit partial sums must carry."""

@@ -198,6 +198,16 @@ __device__ __forceinline__ void codes_segment(float2 (&v)[16], float inv, uint32
 constexpr int kWeightUnroll = 4;         // 32-byte loads in flight per thread in the weight pass
 constexpr int64_t kMaxWeightCtas = 592;  // four CTAs for each of a B200's 148 SMs
 
+// A thread's row within its CTA is tid / L for the L segment threads of a row. The kernels take
+// it as (tid * row_mul) >> kRowShift with row_mul = ceil(2^20 / L). For tid < 2^10 and L <= 2^9
+// the product stays below 2^30 and exceeds tid * 2^20 / L by less than tid < 2^10, while
+// tid * 2^20 / L lies at least 2^20 / L >= 2^11 below the next multiple of 2^20, so the shift
+// gives the exact quotient. It replaces a runtime integer division (a reciprocal, two conversions
+// and corrections) that every thread paid once.
+constexpr int kRowShift = 20;
+
+int row_multiplier(int L) { return static_cast<int>(((1 << kRowShift) + L - 1) / L); }
+
 // Weight pass over `count` cooperating threads, thread `idx` of them.
 __device__ __forceinline__ void weight_pass_threads(const PrologueArgs& a, int64_t idx, int64_t count) {
   for (int seg = 0; seg < a.num_w; ++seg) {
@@ -242,7 +252,7 @@ __device__ __forceinline__ void weight_pass(const PrologueArgs& a, int64_t cta, 
 // CTAs [0, row_ctas) quantize activation rows, the rest run the weight pass.
 template <int LANES, bool VEC32, int MAXT, int MINB>
 __global__ void __launch_bounds__(MAXT, MINB)
-    prologue_kernel(const PrologueArgs a, const int rows_per_cta, const int row_ctas) {
+    prologue_kernel(const PrologueArgs a, const int rows_per_cta, const int row_ctas, const int row_mul) {
   if (gated_out(a.gate, a.bits_table, a.gate_index)) return;
   if (static_cast<int>(blockIdx.x) >= row_ctas) {
     weight_pass(a, blockIdx.x - row_ctas, gridDim.x - row_ctas);
@@ -250,7 +260,7 @@ __global__ void __launch_bounds__(MAXT, MINB)
   }
   const int L = a.Kp >> 5;                       // 32-channel segments per row
   const int tid = threadIdx.x;
-  const int r_local = tid / L;
+  const int r_local = (tid * row_mul) >> kRowShift;   // tid / L (see row_multiplier)
   const int seg = tid - r_local * L;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + r_local;
   const bool active = r_local < rows_per_cta && row < a.M;
@@ -387,7 +397,7 @@ __device__ __forceinline__ void codes_segment64(float2 (&v)[32], float inv, uint
 // owns rows_per_cta rows of Kp / 64 threads each; CTAs [row_ctas, gridDim) run the weight pass.
 template <bool N128, bool VEC32, int MAXT, int MINB>
 __global__ void __launch_bounds__(MAXT, MINB)
-    prologue64_kernel(const PrologueArgs a, const int rows_per_cta, const int row_ctas) {
+    prologue64_kernel(const PrologueArgs a, const int rows_per_cta, const int row_ctas, const int row_mul) {
   if (gated_out(a.gate, a.bits_table, a.gate_index)) return;
   if (static_cast<int>(blockIdx.x) >= row_ctas) {
     weight_pass(a, blockIdx.x - row_ctas, gridDim.x - row_ctas);
@@ -395,7 +405,7 @@ __global__ void __launch_bounds__(MAXT, MINB)
   }
   const int L = a.Kp >> 6;                       // 64-channel segments per row
   const int tid = threadIdx.x;
-  const int r_local = tid / L;
+  const int r_local = (tid * row_mul) >> kRowShift;   // tid / L (see row_multiplier)
   const int seg = tid - r_local * L;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + r_local;
   const bool active = r_local < rows_per_cta && row < a.M;
@@ -585,7 +595,7 @@ __device__ __forceinline__ void nvfp4_weight_pass(const Nvfp4PrologueArgs& a, in
 
 template <int LANES, int MAXT, int MINB>
 __global__ void __launch_bounds__(MAXT, MINB)
-    prologue_nvfp4_kernel(const Nvfp4PrologueArgs a, const int rows_per_cta, const int row_ctas) {
+    prologue_nvfp4_kernel(const Nvfp4PrologueArgs a, const int rows_per_cta, const int row_ctas, const int row_mul) {
   if (gated_out(a.gate, a.gate_table, a.gate_index)) return;
   // CTAs [0, weight_ctas) convert the weights (each loops over several quads, so they start
   // first), the rest quantize activation rows
@@ -597,7 +607,7 @@ __global__ void __launch_bounds__(MAXT, MINB)
   const int row_block = static_cast<int>(blockIdx.x) - weight_ctas;
   const int L = a.Kp >> 5;
   const int tid = threadIdx.x;
-  const int r_local = tid / L;
+  const int r_local = (tid * row_mul) >> kRowShift;   // tid / L (see row_multiplier)
   const int seg = tid - r_local * L;
   const int64_t row = static_cast<int64_t>(row_block) * rows_per_cta + r_local;
   const bool active = r_local < rows_per_cta && row < a.M;
@@ -1001,11 +1011,11 @@ cudaError_t launch_prologue64(const PrologueArgs& a, int64_t w_bytes, cudaStream
   cfg.numAttrs = use_pdl() ? 1 : 0;
   const int rc = static_cast<int>(row_ctas);
   if (a.n == 64) {
-    if (vec32) return cudaLaunchKernelEx(&cfg, prologue64_kernel<false, true, k64Threads, k64MinBlocks>, a, R, rc);
-    return cudaLaunchKernelEx(&cfg, prologue64_kernel<false, false, k64Threads, k64MinBlocks>, a, R, rc);
+    if (vec32) return cudaLaunchKernelEx(&cfg, prologue64_kernel<false, true, k64Threads, k64MinBlocks>, a, R, rc, row_multiplier(L));
+    return cudaLaunchKernelEx(&cfg, prologue64_kernel<false, false, k64Threads, k64MinBlocks>, a, R, rc, row_multiplier(L));
   }
-  if (vec32) return cudaLaunchKernelEx(&cfg, prologue64_kernel<true, true, k64Threads, k64MinBlocks>, a, R, rc);
-  return cudaLaunchKernelEx(&cfg, prologue64_kernel<true, false, k64Threads, k64MinBlocks>, a, R, rc);
+  if (vec32) return cudaLaunchKernelEx(&cfg, prologue64_kernel<true, true, k64Threads, k64MinBlocks>, a, R, rc, row_multiplier(L));
+  return cudaLaunchKernelEx(&cfg, prologue64_kernel<true, false, k64Threads, k64MinBlocks>, a, R, rc, row_multiplier(L));
 }
 
 }  // namespace
@@ -1054,15 +1064,15 @@ cudaError_t launch_prologue_nvfp4(const Nvfp4PrologueArgs& a, cudaStream_t strea
   cfg.numAttrs = use_pdl() ? 1 : 0;
   const int rc = static_cast<int>(row_ctas);
   if (small) {
-    if (a.n == 64) return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<2, kSmallThreads, 4>, a, R, rc);
-    return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<4, kSmallThreads, 4>, a, R, rc);
+    if (a.n == 64) return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<2, kSmallThreads, 4>, a, R, rc, row_multiplier(L));
+    return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<4, kSmallThreads, 4>, a, R, rc, row_multiplier(L));
   }
   if (mid) {
-    if (a.n == 64) return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<2, kMidThreads, 3>, a, R, rc);
-    return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<4, kMidThreads, 3>, a, R, rc);
+    if (a.n == 64) return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<2, kMidThreads, 3>, a, R, rc, row_multiplier(L));
+    return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<4, kMidThreads, 3>, a, R, rc, row_multiplier(L));
   }
-  if (a.n == 64) return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<2, kMaxThreads, 1>, a, R, rc);
-  return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<4, kMaxThreads, 1>, a, R, rc);
+  if (a.n == 64) return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<2, kMaxThreads, 1>, a, R, rc, row_multiplier(L));
+  return cudaLaunchKernelEx(&cfg, prologue_nvfp4_kernel<4, kMaxThreads, 1>, a, R, rc, row_multiplier(L));
 }
 
 cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
@@ -1125,18 +1135,18 @@ cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
   const int rc = static_cast<int>(row_ctas);
   if (small) {
     if (a.n == 64) {
-      if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<2, true, kSmallThreads, 4>, a, R, rc);
-      return cudaLaunchKernelEx(&cfg, prologue_kernel<2, false, kSmallThreads, 4>, a, R, rc);
+      if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<2, true, kSmallThreads, 4>, a, R, rc, row_multiplier(L));
+      return cudaLaunchKernelEx(&cfg, prologue_kernel<2, false, kSmallThreads, 4>, a, R, rc, row_multiplier(L));
     }
-    if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<4, true, kSmallThreads, 4>, a, R, rc);
-    return cudaLaunchKernelEx(&cfg, prologue_kernel<4, false, kSmallThreads, 4>, a, R, rc);
+    if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<4, true, kSmallThreads, 4>, a, R, rc, row_multiplier(L));
+    return cudaLaunchKernelEx(&cfg, prologue_kernel<4, false, kSmallThreads, 4>, a, R, rc, row_multiplier(L));
   }
   if (a.n == 64) {
-    if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<2, true, kMaxThreads, 1>, a, R, rc);
-    return cudaLaunchKernelEx(&cfg, prologue_kernel<2, false, kMaxThreads, 1>, a, R, rc);
+    if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<2, true, kMaxThreads, 1>, a, R, rc, row_multiplier(L));
+    return cudaLaunchKernelEx(&cfg, prologue_kernel<2, false, kMaxThreads, 1>, a, R, rc, row_multiplier(L));
   }
-  if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<4, true, kMaxThreads, 1>, a, R, rc);
-  return cudaLaunchKernelEx(&cfg, prologue_kernel<4, false, kMaxThreads, 1>, a, R, rc);
+  if (vec32) return cudaLaunchKernelEx(&cfg, prologue_kernel<4, true, kMaxThreads, 1>, a, R, rc, row_multiplier(L));
+  return cudaLaunchKernelEx(&cfg, prologue_kernel<4, false, kMaxThreads, 1>, a, R, rc, row_multiplier(L));
 }
 
 }  // namespace tasq

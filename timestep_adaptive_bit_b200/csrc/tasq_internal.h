@@ -114,7 +114,7 @@ enum class OutKind : int { F16 = 0, BF16 = 1, S32 = 2 };
 // DMPQ precision predictor: Gamma = ||out - in||_1 / ||in||_1 over FP16 [M, D] (D % 8 == 0,
 // rows 16-byte aligned), then table[entries[i]] = Gamma > tau ? bits_unstable : bits_stable.
 constexpr int kDmpqMaxEntries = 32;
-constexpr int kDmpqCtasPerSm = 4;
+constexpr int kDmpqCtasPerSm = 2;
 struct DmpqArgs {
   const void* in;
   const void* out;
