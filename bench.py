@@ -347,7 +347,7 @@ def setup_workload(T, torch, wl, device, out_dtype, gemm_mode=0, mask_mode=0, pr
     return ctx, xs, ys
 
 
-def time_dmpq(T, torch, ctx, wl, xs, ys, stream, reps: int = 20):
+def time_dmpq(T, torch, ctx, wl, xs, ys, stream, reps: int = 100):
     """CUDA-event time of tasq_dmpq_update on the block's first input and last output (same
     width). It reads both tensors once: algorithmic bytes 2 * M * D * 2."""
     D_in = wl.block_layers[0][1]
@@ -369,7 +369,8 @@ def time_dmpq(T, torch, ctx, wl, xs, ys, stream, reps: int = 20):
     e1.record(stream)
     torch.cuda.synchronize()
     us = 1e3 * e0.elapsed_time(e1) / reps
-    return {"us": us, "gbs": 4.0 * M * D_in / (us * 1e-6) / 1e9, "shape": [M, D_in], "gamma": float(g.item())}
+    return {"us": us, "gbs": 4.0 * M * D_in / (us * 1e-6) / 1e9, "shape": [M, D_in], "calls": reps,
+            "gamma": float(g.item())}
 
 
 # threshold of the on-device predictor of dmpq_online workloads, set once per run
@@ -941,7 +942,7 @@ def main(argv=None):
         "dmpq_predictor": None if dmpq is None else {
             "bound": "hbm", "achieved": dmpq["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": dmpq["gbs"] / peaks["hbm_gbs"], "us_per_call": dmpq["us"], "shape": dmpq["shape"],
-            "gamma": dmpq["gamma"]},
+            "calls": dmpq["calls"], "gamma": dmpq["gamma"]},
     }
     print(json.dumps(line), flush=True)
     return 0 if status == 0 else 1
